@@ -1,0 +1,218 @@
+/*
+ * pagedattn.h -- C ABI of libpagedattn: paged-attention decode on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation (gllm PR #116 "feat(backend): sliding-window
+ * PagedAttention", section "What changes", Interface):
+ *
+ *   PagedAttention(dst, q, kCache, vCache, blockTables, seqLens, queryLens,
+ *                  scale, window)
+ *
+ * For every row b with queryLens[b] = L > 0, every query token i < L and every
+ * query head h:
+ *   p   = seqLens[b] - L + i          (the L new tokens are the last L of
+ *                                      the row's seqLens[b] cached tokens)
+ *   lo  = window > 0 ? max(0, p + 1 - window) : 0,   hi = p + 1
+ *   g   = h / (H_q / H_kv)            (grouped-query heads; ExecuTorch PR
+ *                                      #18759, sdpa_decode_splitk docstring)
+ *   k_t = kCache[blockTables[b][t / BS]][g][t % BS][:]   (same for v_t)
+ *   dst[b,i,h,:] = sum_{t in [lo,hi)} softmax_t(scale * q[b,i,h,:] . k_t) v_t
+ *
+ * Long spans are cut into split-K partitions whose partial results are merged
+ * by a log-sum-exp reduce (ExecuTorch PR #18759, split-K flash-decoding and
+ * its reduce kernel); when one partition suffices the kernel writes dst
+ * directly and needs no temporaries (aiter PR #2914 "Pa gluon swa mtp opt",
+ * the one_shot path).
+ *
+ * Layouts (all row-major, element type bf16 unless noted):
+ *   q, dst        [sum(queryLens)][H_q][head_dim], rows packed in batch order
+ *   kCache,vCache [num_blocks][H_kv][kvBlockSize][head_dim]
+ *   blockTables   int32 [batch][max_blocks_per_seq]; only the first
+ *                 ceil(seqLens[b] / kvBlockSize) entries of row b are read
+ *   seqLens, queryLens, windows  int32 [batch]
+ *
+ * Ownership: the caller owns every buffer, including the workspace; the
+ * library allocates no device memory in pa_decode.  All calls are
+ * asynchronous on the given stream (a cudaStream_t passed as void*, NULL for
+ * the legacy default stream) except where stated.
+ *
+ * Errors: every entry point returns PA_OK or a PA_ERR_* code and leaves a
+ * one-line message for pa_last_error().  Conditions only the device can see
+ * (a row with queryLen > seqLen, a block-table entry outside the pool, a
+ * length beyond the caller's hints, a wait that timed out) skip the affected
+ * work and set bits in a device status word read by pa_device_status().
+ */
+#ifndef PAGEDATTN_H
+#define PAGEDATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes. */
+#define PA_OK 0
+#define PA_ERR_ARG 1          /* invalid argument (null pointer, bad size, misalignment) */
+#define PA_ERR_UNSUPPORTED 2  /* valid but not built: head_dim or block size */
+#define PA_ERR_WORKSPACE 3    /* workspace missing or smaller than pa_workspace_size */
+#define PA_ERR_CUDA 4         /* a CUDA runtime call failed */
+
+/* Device status bits (pa_device_status). */
+#define PA_DEV_TIMEOUT 1u     /* a pipeline wait gave up after ~1 s */
+#define PA_DEV_BAD_ROW 2u     /* queryLens[b] > seqLens[b], negative length or window */
+#define PA_DEV_BAD_BLOCK 4u   /* a block-table entry outside [0, num_blocks) */
+#define PA_DEV_HINT 8u        /* a row longer than max_span_hint / max_query_len_hint */
+
+/* Kernel variants (pa_params.force_variant, pa_plan_info.variant). */
+#define PA_VARIANT_AUTO 0
+#define PA_VARIANT_FMA 1      /* CUDA-core FMA scores and PV (few rows per kv head) */
+
+typedef struct pa_params {
+    int batch;               /* rows */
+    int num_q_heads;         /* H_q, a multiple of num_kv_heads */
+    int num_kv_heads;        /* H_kv */
+    int head_dim;            /* 64 or 128 */
+    int num_blocks;          /* KV pool size in blocks */
+    int max_blocks_per_seq;  /* blockTables row stride (entries) */
+    /* Host hints.  max_span_hint >= max_b union span, where a row's union
+     * span is seqLen - max(0, seqLen - queryLen + 1 - window) for window > 0
+     * and seqLen otherwise; max_query_len_hint >= max_b queryLens[b].  With
+     * both set pa_decode never synchronises.  0 means unknown: pa_decode then
+     * copies the lengths to the host once (a stream synchronisation). */
+    int max_span_hint;
+    int max_query_len_hint;
+    const int32_t *windows;  /* device [batch] per-row windows, or NULL for the scalar window */
+    void *workspace;         /* device, >= pa_workspace_size() bytes when that is > 0 */
+    size_t workspace_bytes;
+    int force_variant;       /* PA_VARIANT_AUTO, or a PA_VARIANT_* for tests and A/B runs */
+    int force_partitions;    /* 0 = dispatcher's choice; n > 0 cuts the longest span into ~n partitions */
+} pa_params;
+
+/* What the dispatcher chose for a call (pa_plan). */
+typedef struct pa_plan_info {
+    int variant;             /* PA_VARIANT_* */
+    int partition_tokens;    /* tokens per split-K partition (multiple of 64) */
+    int max_partitions;      /* partitions of the longest span (1 = one-shot) */
+    int one_shot;            /* 1: every row fits one partition, no workspace, no reduce */
+    int max_rows;            /* rows per (row, kv head) unit: (H_q/H_kv) * max queryLen */
+    int slab_rows;           /* rows one CTA handles; units with more rows use several CTAs */
+    int consumer_warps;      /* compute warps per CTA (plus one copy warp) */
+    int stages;              /* shared-memory pipeline depth */
+    int grid_x, grid_y, grid_z;
+    int block_threads;
+    size_t smem_bytes;
+    size_t workspace_bytes;  /* 0 when one_shot */
+    int num_sms, ctas_per_sm;
+} pa_plan_info;
+
+/*
+ * pa_decode -- paged-attention decode (the operation at the top of this file).
+ *
+ *   dst          device bf16 [sum(queryLens)][H_q][head_dim], written for rows
+ *                with queryLens[b] > 0; other memory is untouched
+ *   q            device bf16 [sum(queryLens)][H_q][head_dim]
+ *   kCache,vCache device bf16 [num_blocks][H_kv][kvBlockSize][head_dim]
+ *   blockTables  device int32 [batch][max_blocks_per_seq]
+ *   seqLens      device int32 [batch], cached tokens per row (includes the new ones)
+ *   queryLens    device int32 [batch], new query tokens per row (0 skips the row)
+ *   scale        multiplies q.k, used exactly as given
+ *   window       0 = full causal; w > 0 = each token sees its last w positions;
+ *                overridden per row by params->windows when that is not NULL
+ *   kvBlockSize  tokens per KV block: a power of two in [16, 1024]
+ *   params       dimensions, hints, workspace (see pa_params)
+ *   stream       cudaStream_t
+ *
+ * All device pointers must be 16-byte aligned.  Returns PA_ERR_ARG for null
+ * pointers, H_q % H_kv != 0, negative window or hints, misalignment;
+ * PA_ERR_UNSUPPORTED for head_dim not in {64,128} or a block size outside
+ * the set above; PA_ERR_WORKSPACE when split-K partials are needed and the
+ * workspace is too small; PA_ERR_CUDA when a launch fails.
+ */
+int pa_decode(void *dst, const void *q, const void *kCache, const void *vCache,
+              const int32_t *blockTables, const int32_t *seqLens,
+              const int32_t *queryLens, float scale, int window, int kvBlockSize,
+              const pa_params *params, void *stream);
+
+/*
+ * pa_workspace_size -- bytes of workspace pa_decode needs for these params
+ * (split-K partial maxima/sums and outputs for max(1, P) partitions, the
+ * allocation rule aiter PR #2914's review asks for).  Uses the hints; with a
+ * zero span hint it assumes the longest row fills max_blocks_per_seq blocks.
+ * Returns 0 when the call is one-shot; (size_t)-1 on invalid params.
+ * Host only; needs a CUDA device only when num_sms is not fixed (it queries
+ * the current device's SM count and occupancy).
+ */
+size_t pa_workspace_size(const pa_params *params, int kvBlockSize);
+
+/*
+ * pa_plan -- the dispatcher's decision for these params, without launching.
+ * num_sms / ctas_per_sm: 0 queries the current device; > 0 fixes them
+ * (host-only use, e.g. on a machine without a GPU).  Host only.
+ */
+int pa_plan(const pa_params *params, int kvBlockSize, int num_sms, int ctas_per_sm,
+            pa_plan_info *out);
+
+/*
+ * pa_visible_ranges -- the [lo, hi) each query token sees (section "What
+ * changes" of the gllm page: max(0, end - window) .. end), computed on the
+ * device with the same span function the kernels use.
+ *   lo, hi       device int32 [sum(queryLens)], packed in batch order
+ *   seqLens, queryLens, windows (may be NULL)  device int32 [batch]
+ * Returns PA_ERR_ARG for null outputs/lengths, batch < 0 or window < 0.
+ */
+int pa_visible_ranges(int32_t *lo, int32_t *hi, const int32_t *seqLens,
+                      const int32_t *queryLens, int window, const int32_t *windows,
+                      int batch, void *stream);
+
+/*
+ * pa_decode_host -- end-to-end call with host buffers: copies q, blockTables,
+ * seqLens, queryLens (and windows) from host memory into the caller's
+ * workspace, runs pa_decode, copies dst back, and synchronises the stream.
+ * The KV caches stay on the device (they are resident state).  Host buffers
+ * should be pinned for asynchronous copies.
+ *   dst_host, q_host  host bf16 [sum(queryLens)][H_q][head_dim]
+ *   blockTables_host, seqLens_host, queryLens_host  host int32
+ *   params->windows   host int32 [batch] or NULL (host memory in this call)
+ *   params->workspace device, >= pa_host_workspace_size() bytes
+ * Hints are computed from the host lengths and need not be set.
+ */
+int pa_decode_host(void *dst_host, const void *q_host, const void *kCache,
+                   const void *vCache, const int32_t *blockTables_host,
+                   const int32_t *seqLens_host, const int32_t *queryLens_host,
+                   float scale, int window, int kvBlockSize, const pa_params *params,
+                   void *stream);
+
+/* Workspace bytes pa_decode_host needs (staging for q, dst and the tables,
+ * plus the split-K workspace); (size_t)-1 on invalid params. */
+size_t pa_host_workspace_size(const pa_params *params, int kvBlockSize, int window,
+                              const int32_t *seqLens_host, const int32_t *queryLens_host);
+
+/*
+ * pa_extents_host -- the two hints pa_params takes, from host copies of the
+ * lengths: *max_span = longest union span over rows with queryLen > 0 (the
+ * row's visible positions [max(0, S-L+1-window), S) for window > 0, else
+ * [0, S)), *max_query_len = longest queryLen.  windows may be NULL (scalar
+ * window).  Returns PA_ERR_ARG on a row with queryLen > seqLen or a negative
+ * length or window.  Host only.
+ */
+int pa_extents_host(const int32_t *seqLens, const int32_t *queryLens,
+                    const int32_t *windows, int window, int batch, int *max_span,
+                    int *max_query_len);
+
+/* Reads the device status word (PA_DEV_* bits) of the current device into
+ * *status and clears it when clear != 0.  Synchronises the stream. */
+int pa_device_status(unsigned int *status, int clear, void *stream);
+
+/* Message of the last error on this thread ("" after success). */
+const char *pa_last_error(void);
+
+/* Library version string. */
+const char *pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDATTN_H */

@@ -1,0 +1,456 @@
+// pa_api.cu -- host side of libpagedattn: the C ABI declared in
+// include/pagedattn.h, argument validation, and the dispatcher that picks the
+// split-K partition size, kernel variant and grid.
+//
+// Dispatcher rule.  gllm PR #116 "feat(backend): sliding-window
+// PagedAttention" ("What changes", CUDA): the launcher sizes its work from the
+// longest *windowed* span, not the longest context.  ExecuTorch PR #18759
+// (review suggestion 6) notes that a fixed 256-tokens-per-split rule ignores
+// the SM count.  Here the partition size comes from the longest windowed span,
+// the number of (row, kv head) units and the SMs x resident CTAs of the
+// chosen kernel: few units get one balanced wave of partitions, many units
+// get about four waves so ragged rows even out.  One partition per row means
+// the one-shot path: the kernel writes dst itself, with no workspace and no
+// reduce (aiter PR #2914 "Pa gluon swa mtp opt", one_shot).
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/pagedattn.h"
+#include "pa_kernels.cuh"
+#include "pa_span.h"
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+int succeed() {
+  g_err.clear();
+  return PA_OK;
+}
+
+constexpr int TS = pa::kStageTokens;
+constexpr int kMinPartTokens = 256;
+
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+int ilog2(int x) {
+  int s = 0;
+  while ((1 << s) < x) ++s;
+  return s;
+}
+
+long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int current_sms(int* out) {
+  static std::mutex mu;
+  static std::vector<int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(PA_ERR_CUDA, "cudaGetDevice failed");
+  std::lock_guard<std::mutex> lock(mu);
+  if ((int)cache.size() <= dev) cache.resize(dev + 1, 0);
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      return fail(PA_ERR_CUDA, "cannot read the SM count of device %d", dev);
+    cache[dev] = n;
+  }
+  *out = cache[dev];
+  return PA_OK;
+}
+
+int check_params(const pa_params* p, int bs) {
+  if (!p) return fail(PA_ERR_ARG, "params is NULL");
+  if (p->batch < 0 || p->batch > 65535)
+    return fail(PA_ERR_ARG, "batch %d outside [0, 65535]", p->batch);
+  if (p->num_q_heads <= 0 || p->num_kv_heads <= 0 || p->num_kv_heads > 65535)
+    return fail(PA_ERR_ARG, "head counts must be positive (H_q=%d, H_kv=%d)", p->num_q_heads,
+                p->num_kv_heads);
+  if (p->num_q_heads % p->num_kv_heads != 0)
+    return fail(PA_ERR_ARG, "H_q=%d is not a multiple of H_kv=%d", p->num_q_heads,
+                p->num_kv_heads);
+  if (p->head_dim != 64 && p->head_dim != 128)
+    return fail(PA_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", p->head_dim);
+  if (!is_pow2(bs) || bs < 16 || bs > 1024)
+    return fail(PA_ERR_UNSUPPORTED, "kvBlockSize %d not supported (power of two in [16,1024])", bs);
+  if (p->num_blocks <= 0 || p->max_blocks_per_seq <= 0)
+    return fail(PA_ERR_ARG, "num_blocks and max_blocks_per_seq must be positive");
+  if ((long long)p->max_blocks_per_seq * bs > (long long)INT32_MAX)
+    return fail(PA_ERR_ARG, "max_blocks_per_seq * kvBlockSize overflows int32");
+  if (p->max_span_hint < 0 || p->max_query_len_hint < 0)
+    return fail(PA_ERR_ARG, "hints must be >= 0");
+  if (p->force_partitions < 0) return fail(PA_ERR_ARG, "force_partitions must be >= 0");
+  if (p->force_variant != PA_VARIANT_AUTO && p->force_variant != PA_VARIANT_FMA)
+    return fail(PA_ERR_ARG, "unknown force_variant %d", p->force_variant);
+  return PA_OK;
+}
+
+struct Plan {
+  pa_plan_info info;
+  pa::KernelShape shape;
+  size_t lse_bytes, o_bytes;
+};
+
+// span: longest union span over rows; qlen: longest queryLen.
+int make_plan(const pa_params* p, int bs, int span, int qlen, int num_sms, int ctas_per_sm,
+              Plan* out) {
+  Plan pl;
+  memset(&pl, 0, sizeof pl);
+  const int G = p->num_q_heads / p->num_kv_heads;
+  span = std::max(span, 1);
+  qlen = std::max(qlen, 1);
+  if ((long long)G * qlen > 4096)
+    return fail(PA_ERR_UNSUPPORTED, "rows per kv head %lld exceed 4096", (long long)G * qlen);
+  const int rmax = G * qlen;
+  const int ncw = rmax <= 16 ? 4 : 8;
+  const int slab_rows = 4 * ncw;
+  const int nslab = (int)cdiv(rmax, slab_rows);
+  pl.shape.head_dim = p->head_dim;
+  pl.shape.consumer_warps = ncw;
+  pl.shape.stages = p->head_dim == 128 ? 3 : 4;
+
+  // Partition-size cap: the CTA caches its slice of the block table in smem.
+  const int cap = std::max(TS, ((pa::kMaxTableCache - 2) * bs) / TS * TS);
+  const size_t smem_max = pa::fma_smem_bytes(p->head_dim, pl.shape.stages, cap, bs);
+  if (num_sms <= 0) {
+    int rc = current_sms(&num_sms);
+    if (rc) return rc;
+  }
+  if (ctas_per_sm <= 0) {
+    ctas_per_sm = pa::occupancy_partition_fma(pl.shape, smem_max);
+    if (ctas_per_sm <= 0)
+      return fail(PA_ERR_CUDA, "occupancy query failed: %s", cudaGetErrorString(cudaGetLastError()));
+  }
+  const long long units = (long long)p->batch * p->num_kv_heads * nslab;
+  const long long slots = (long long)num_sms * ctas_per_sm;
+
+  long long ptok;
+  if (p->force_partitions > 0) {
+    ptok = cdiv(cdiv(span, p->force_partitions), TS) * TS;
+  } else {
+    const long long waves = (units * 4 <= slots) ? 1 : 4;
+    const long long want = std::max<long long>(1, cdiv(waves * slots, std::max<long long>(units, 1)));
+    ptok = cdiv(cdiv(span, want), TS) * TS;
+    ptok = std::max<long long>(ptok, kMinPartTokens);
+  }
+  ptok = std::min<long long>(std::max<long long>(ptok, TS), cap);
+  const long long max_parts = cdiv((long long)span + TS - 1, ptok);
+  if (max_parts > (1LL << 30)) return fail(PA_ERR_UNSUPPORTED, "too many partitions");
+
+  pa_plan_info& in = pl.info;
+  in.variant = PA_VARIANT_FMA;
+  in.partition_tokens = (int)ptok;
+  in.max_partitions = (int)max_parts;
+  in.one_shot = max_parts == 1;
+  in.max_rows = rmax;
+  in.slab_rows = slab_rows;
+  in.consumer_warps = ncw;
+  in.stages = pl.shape.stages;
+  in.grid_x = (int)max_parts;
+  in.grid_y = p->num_kv_heads * nslab;
+  in.grid_z = p->batch;
+  in.block_threads = 32 * (ncw + 1);
+  in.smem_bytes = pa::fma_smem_bytes(p->head_dim, pl.shape.stages, (int)ptok, bs);
+  in.num_sms = num_sms;
+  in.ctas_per_sm = ctas_per_sm;
+  if (!in.one_shot) {
+    const size_t partials = (size_t)p->batch * p->num_kv_heads * max_parts * rmax;
+    pl.lse_bytes = align256(partials * sizeof(float));
+    pl.o_bytes = align256(partials * p->head_dim * sizeof(float));
+    in.workspace_bytes = pl.lse_bytes + pl.o_bytes;
+  }
+  *out = pl;
+  return PA_OK;
+}
+
+// Longest union span and query length from host copies of the lengths.
+int host_extents(const int32_t* S, const int32_t* L, const int32_t* W, int window, int batch,
+                 int* span, int* qlen, long long* ntok) {
+  int sp = 0, ql = 0;
+  long long nt = 0;
+  for (int b = 0; b < batch; ++b) {
+    const int w = W ? W[b] : window;
+    if (L[b] < 0 || S[b] < 0 || L[b] > S[b] || w < 0)
+      return fail(PA_ERR_ARG, "row %d: queryLen %d, seqLen %d, window %d are inconsistent", b, L[b],
+                  S[b], w);
+    nt += L[b];
+    if (L[b] == 0) continue;
+    sp = std::max(sp, pa::union_span(S[b], L[b], w));
+    ql = std::max(ql, (int)L[b]);
+  }
+  *span = sp;
+  *qlen = ql;
+  if (ntok) *ntok = nt;
+  return PA_OK;
+}
+
+int device_extents(const pa_params* p, const int32_t* seqLens, const int32_t* queryLens,
+                   int window, cudaStream_t stream, int* span, int* qlen) {
+  const int B = p->batch;
+  std::vector<int32_t> S(B), L(B), W(p->windows ? B : 0);
+  cudaError_t e = cudaMemcpyAsync(S.data(), seqLens, B * sizeof(int32_t), cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(L.data(), queryLens, B * sizeof(int32_t), cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess && p->windows)
+    e = cudaMemcpyAsync(W.data(), p->windows, B * sizeof(int32_t), cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "reading lengths: %s", cudaGetErrorString(e));
+  return host_extents(S.data(), L.data(), p->windows ? W.data() : nullptr, window, B, span, qlen,
+                      nullptr);
+}
+
+int decode_impl(void* dst, const void* q, const void* kCache, const void* vCache,
+                const int32_t* blockTables, const int32_t* seqLens, const int32_t* queryLens,
+                float scale, int window, int bs, const pa_params* p, cudaStream_t stream,
+                int span, int qlen) {
+  Plan pl;
+  int rc = make_plan(p, bs, span, qlen, 0, 0, &pl);
+  if (rc) return rc;
+  const pa_plan_info& in = pl.info;
+  if (!in.one_shot) {
+    if (!p->workspace || p->workspace_bytes < in.workspace_bytes)
+      return fail(PA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", in.workspace_bytes,
+                  p->workspace ? p->workspace_bytes : (size_t)0);
+    if (!aligned16(p->workspace)) return fail(PA_ERR_ARG, "workspace must be 16-byte aligned");
+  }
+  pa::DecodeArgs a;
+  memset(&a, 0, sizeof a);
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k_cache = static_cast<const __nv_bfloat16*>(kCache);
+  a.v_cache = static_cast<const __nv_bfloat16*>(vCache);
+  a.block_tables = blockTables;
+  a.seq_lens = seqLens;
+  a.query_lens = queryLens;
+  a.windows = p->windows;
+  a.dst = static_cast<__nv_bfloat16*>(dst);
+  if (!in.one_shot) {
+    a.ws_lse = static_cast<float*>(p->workspace);
+    a.ws_o = reinterpret_cast<float*>(static_cast<char*>(p->workspace) + pl.lse_bytes);
+  }
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.window = window;
+  a.batch = p->batch;
+  a.num_q_heads = p->num_q_heads;
+  a.num_kv_heads = p->num_kv_heads;
+  a.group = p->num_q_heads / p->num_kv_heads;
+  a.head_dim = p->head_dim;
+  a.block_size = bs;
+  a.block_shift = ilog2(bs);
+  a.max_blocks_per_seq = p->max_blocks_per_seq;
+  a.num_blocks = p->num_blocks;
+  a.part_tokens = in.partition_tokens;
+  a.max_parts = in.max_partitions;
+  a.max_rows = in.max_rows;
+  a.slab_rows = in.slab_rows;
+  a.num_slabs = in.grid_y / p->num_kv_heads;
+
+  const dim3 grid(in.grid_x, in.grid_y, in.grid_z);
+  cudaError_t e = pa::launch_partition_fma(a, pl.shape, grid, in.smem_bytes, stream);
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "partition kernel launch: %s", cudaGetErrorString(e));
+  if (!in.one_shot) {
+    e = pa::launch_reduce(a, stream);
+    if (e != cudaSuccess) return fail(PA_ERR_CUDA, "reduce kernel launch: %s", cudaGetErrorString(e));
+  }
+  if (getenv("PA_LOG_PLAN"))
+    fprintf(stderr,
+            "[pagedattn] variant=%d ptok=%d parts=%d one_shot=%d rows=%d slab=%d warps=%d "
+            "stages=%d grid=(%d,%d,%d) smem=%zu ws=%zu sms=%d ctas/sm=%d\n",
+            in.variant, in.partition_tokens, in.max_partitions, in.one_shot, in.max_rows,
+            in.slab_rows, in.consumer_warps, in.stages, in.grid_x, in.grid_y, in.grid_z,
+            in.smem_bytes, in.workspace_bytes, in.num_sms, in.ctas_per_sm);
+  return succeed();
+}
+
+}  // namespace
+
+extern "C" {
+
+int pa_decode(void* dst, const void* q, const void* kCache, const void* vCache,
+              const int32_t* blockTables, const int32_t* seqLens, const int32_t* queryLens,
+              float scale, int window, int kvBlockSize, const pa_params* params, void* stream) {
+  int rc = check_params(params, kvBlockSize);
+  if (rc) return rc;
+  if (!dst || !q || !kCache || !vCache || !blockTables || !seqLens || !queryLens)
+    return fail(PA_ERR_ARG, "a required pointer is NULL");
+  if (!aligned16(dst) || !aligned16(q) || !aligned16(kCache) || !aligned16(vCache))
+    return fail(PA_ERR_ARG, "dst, q, kCache and vCache must be 16-byte aligned");
+  if (window < 0) return fail(PA_ERR_ARG, "window %d is negative", window);
+  if (!(scale == scale) || scale > 3.0e38f || scale < -3.0e38f)
+    return fail(PA_ERR_ARG, "scale must be finite");
+  if (params->batch == 0) return succeed();
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int span = params->max_span_hint, qlen = params->max_query_len_hint;
+  if (span == 0 || qlen == 0) {
+    rc = device_extents(params, seqLens, queryLens, window, st, &span, &qlen);
+    if (rc) return rc;
+    if (qlen == 0) return succeed();  // every row has queryLen 0
+  }
+  return decode_impl(dst, q, kCache, vCache, blockTables, seqLens, queryLens, scale, window,
+                     kvBlockSize, params, st, span, qlen);
+}
+
+size_t pa_workspace_size(const pa_params* params, int kvBlockSize) {
+  if (check_params(params, kvBlockSize)) return (size_t)-1;
+  const int span = params->max_span_hint > 0 ? params->max_span_hint
+                                             : params->max_blocks_per_seq * kvBlockSize;
+  const int qlen = params->max_query_len_hint > 0 ? params->max_query_len_hint : 1;
+  Plan pl;
+  if (make_plan(params, kvBlockSize, span, qlen, 0, 0, &pl)) return (size_t)-1;
+  succeed();
+  return pl.info.workspace_bytes;
+}
+
+int pa_plan(const pa_params* params, int kvBlockSize, int num_sms, int ctas_per_sm,
+            pa_plan_info* out) {
+  int rc = check_params(params, kvBlockSize);
+  if (rc) return rc;
+  if (!out) return fail(PA_ERR_ARG, "out is NULL");
+  const int span = params->max_span_hint > 0 ? params->max_span_hint
+                                             : params->max_blocks_per_seq * kvBlockSize;
+  const int qlen = params->max_query_len_hint > 0 ? params->max_query_len_hint : 1;
+  Plan pl;
+  rc = make_plan(params, kvBlockSize, span, qlen, num_sms, ctas_per_sm, &pl);
+  if (rc) return rc;
+  *out = pl.info;
+  return succeed();
+}
+
+int pa_visible_ranges(int32_t* lo, int32_t* hi, const int32_t* seqLens, const int32_t* queryLens,
+                      int window, const int32_t* windows, int batch, void* stream) {
+  if (!lo || !hi || !seqLens || !queryLens) return fail(PA_ERR_ARG, "a required pointer is NULL");
+  if (batch < 0) return fail(PA_ERR_ARG, "batch %d is negative", batch);
+  if (window < 0) return fail(PA_ERR_ARG, "window %d is negative", window);
+  if (batch == 0) return succeed();
+  cudaError_t e = pa::launch_ranges(lo, hi, seqLens, queryLens, window, windows, batch,
+                                    static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "ranges kernel launch: %s", cudaGetErrorString(e));
+  return succeed();
+}
+
+size_t pa_host_workspace_size(const pa_params* params, int kvBlockSize, int window,
+                              const int32_t* seqLens_host, const int32_t* queryLens_host) {
+  if (check_params(params, kvBlockSize) || !seqLens_host || !queryLens_host) return (size_t)-1;
+  int span = 0, qlen = 0;
+  long long ntok = 0;
+  if (window < 0) return (size_t)-1;
+  if (host_extents(seqLens_host, queryLens_host, params->windows, window, params->batch, &span,
+                   &qlen, &ntok))
+    return (size_t)-1;
+  const size_t B = params->batch;
+  const size_t qbytes = align256((size_t)ntok * params->num_q_heads * params->head_dim * 2);
+  size_t total = 2 * qbytes + align256(B * params->max_blocks_per_seq * 4) + 3 * align256(B * 4);
+  if (qlen > 0) {
+    Plan pl;
+    if (make_plan(params, kvBlockSize, span, qlen, 0, 0, &pl)) return (size_t)-1;
+    total += pl.info.workspace_bytes;
+  }
+  succeed();
+  return total;
+}
+
+int pa_decode_host(void* dst_host, const void* q_host, const void* kCache, const void* vCache,
+                   const int32_t* blockTables_host, const int32_t* seqLens_host,
+                   const int32_t* queryLens_host, float scale, int window, int kvBlockSize,
+                   const pa_params* params, void* stream) {
+  int rc = check_params(params, kvBlockSize);
+  if (rc) return rc;
+  if (!dst_host || !q_host || !kCache || !vCache || !blockTables_host || !seqLens_host ||
+      !queryLens_host)
+    return fail(PA_ERR_ARG, "a required pointer is NULL");
+  if (window < 0) return fail(PA_ERR_ARG, "window %d is negative", window);
+  if (!aligned16(kCache) || !aligned16(vCache))
+    return fail(PA_ERR_ARG, "kCache and vCache must be 16-byte aligned");
+  const int B = params->batch;
+  if (B == 0) return succeed();
+  int span = 0, qlen = 0;
+  long long ntok = 0;
+  rc = host_extents(seqLens_host, queryLens_host, params->windows, window, B, &span, &qlen, &ntok);
+  if (rc) return rc;
+  const size_t need =
+      pa_host_workspace_size(params, kvBlockSize, window, seqLens_host, queryLens_host);
+  if (need == (size_t)-1) return fail(PA_ERR_ARG, "%s", g_err.c_str());
+  if (!params->workspace || params->workspace_bytes < need)
+    return fail(PA_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need,
+                params->workspace ? params->workspace_bytes : (size_t)0);
+  if (!aligned16(params->workspace)) return fail(PA_ERR_ARG, "workspace must be 16-byte aligned");
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(params->workspace);
+  const size_t qbytes_raw = (size_t)ntok * params->num_q_heads * params->head_dim * 2;
+  const size_t qbytes = align256(qbytes_raw);
+  const size_t btbytes = (size_t)B * params->max_blocks_per_seq * 4;
+  char* d_q = ws;
+  char* d_dst = d_q + qbytes;
+  char* d_bt = d_dst + qbytes;
+  char* d_S = d_bt + align256(btbytes);
+  char* d_L = d_S + align256((size_t)B * 4);
+  char* d_W = d_L + align256((size_t)B * 4);
+  char* d_split = d_W + align256((size_t)B * 4);
+
+  cudaError_t e = cudaSuccess;
+  if (qbytes_raw) e = cudaMemcpyAsync(d_q, q_host, qbytes_raw, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(d_bt, blockTables_host, btbytes, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(d_S, seqLens_host, (size_t)B * 4, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(d_L, queryLens_host, (size_t)B * 4, cudaMemcpyHostToDevice, st);
+  if (e == cudaSuccess && params->windows)
+    e = cudaMemcpyAsync(d_W, params->windows, (size_t)B * 4, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "host-to-device copy: %s", cudaGetErrorString(e));
+
+  if (qlen > 0) {
+    pa_params dp = *params;
+    dp.windows = params->windows ? reinterpret_cast<const int32_t*>(d_W) : nullptr;
+    dp.workspace = d_split;
+    dp.workspace_bytes = params->workspace_bytes - (size_t)(d_split - ws);
+    dp.max_span_hint = span;
+    dp.max_query_len_hint = qlen;
+    rc = decode_impl(d_dst, d_q, kCache, vCache, reinterpret_cast<const int32_t*>(d_bt),
+                     reinterpret_cast<const int32_t*>(d_S), reinterpret_cast<const int32_t*>(d_L),
+                     scale, window, kvBlockSize, &dp, st, span, qlen);
+    if (rc) return rc;
+  }
+  if (qbytes_raw) e = cudaMemcpyAsync(dst_host, d_dst, qbytes_raw, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "device-to-host copy: %s", cudaGetErrorString(e));
+  return succeed();
+}
+
+int pa_extents_host(const int32_t* seqLens, const int32_t* queryLens, const int32_t* windows,
+                    int window, int batch, int* max_span, int* max_query_len) {
+  if (!seqLens || !queryLens || !max_span || !max_query_len)
+    return fail(PA_ERR_ARG, "a required pointer is NULL");
+  if (batch < 0 || window < 0) return fail(PA_ERR_ARG, "batch and window must be >= 0");
+  int rc = host_extents(seqLens, queryLens, windows, window, batch, max_span, max_query_len, nullptr);
+  if (rc) return rc;
+  return succeed();
+}
+
+int pa_device_status(unsigned int* status, int clear, void* stream) {
+  if (!status) return fail(PA_ERR_ARG, "status is NULL");
+  cudaError_t e = pa::read_status(status, clear != 0, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "reading status: %s", cudaGetErrorString(e));
+  return succeed();
+}
+
+const char* pa_last_error(void) { return g_err.c_str(); }
+
+const char* pa_version(void) { return "libpagedattn 0.1 (sm_100a)"; }
+
+}  // extern "C"

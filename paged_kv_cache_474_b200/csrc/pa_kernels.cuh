@@ -1,0 +1,66 @@
+// pa_kernels.cuh -- launch interface between the host dispatcher (pa_api.cu)
+// and the sm_100a kernels (pa_partition.cu, pa_reduce.cu).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace pa {
+
+constexpr int kStageTokens = 64;  // tokens per shared-memory pipeline stage
+constexpr int kMaxTableCache = 1024;  // block-table entries a CTA caches in smem
+
+// Everything a decode launch needs; passed by value as a __grid_constant__.
+struct DecodeArgs {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k_cache;
+  const __nv_bfloat16* v_cache;
+  const int32_t* block_tables;
+  const int32_t* seq_lens;
+  const int32_t* query_lens;
+  const int32_t* windows;  // may be null
+  __nv_bfloat16* dst;
+  float* ws_lse;  // [B][H_kv][max_parts][max_rows]  log2-domain lse of each partial
+  float* ws_o;    // [B][H_kv][max_parts][max_rows][D] normalised partial outputs
+  float scale_log2;  // scale * log2(e): scores are kept in the log2 domain
+  int window;
+  int batch, num_q_heads, num_kv_heads, group, head_dim;
+  int block_size, block_shift, max_blocks_per_seq, num_blocks;
+  int part_tokens;  // tokens per partition, a multiple of kStageTokens
+  int max_parts;    // partitions per unit the workspace holds (1 = one-shot)
+  int max_rows;     // rows per unit the workspace holds
+  int slab_rows;    // rows one CTA handles
+  int num_slabs;    // CTAs per unit along grid.y (grid.y = H_kv * num_slabs)
+};
+
+// Compile-time shape of a partition-kernel instance.
+struct KernelShape {
+  int head_dim;
+  int consumer_warps;
+  int stages;
+};
+
+// Dynamic shared memory of the FMA partition kernel.
+size_t fma_smem_bytes(int head_dim, int stages, int part_tokens, int block_size);
+
+// Launches the FMA partition kernel; returns the launch error.
+cudaError_t launch_partition_fma(const DecodeArgs& a, const KernelShape& k, dim3 grid,
+                                 size_t smem, cudaStream_t stream);
+
+// Occupancy (CTAs per SM) of an FMA partition-kernel instance.
+int occupancy_partition_fma(const KernelShape& k, size_t smem);
+
+// Launches the log-sum-exp reduce over (rows, kv heads, batch).
+cudaError_t launch_reduce(const DecodeArgs& a, cudaStream_t stream);
+
+// Launches the visible-range kernel.
+cudaError_t launch_ranges(int32_t* lo, int32_t* hi, const int32_t* seq_lens,
+                          const int32_t* query_lens, int window, const int32_t* windows,
+                          int batch, cudaStream_t stream);
+
+// Reads (and optionally clears) the device status word.
+cudaError_t read_status(unsigned int* status, bool clear, cudaStream_t stream);
+
+}  // namespace pa

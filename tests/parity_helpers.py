@@ -1,0 +1,107 @@
+"""Helpers shared by the GPU parity tests: host copies for the oracle,
+sub-problems for sampled checks at full size, and the tolerance check.
+
+Tolerance (reading of "max-abs 2e-2 and rel 2e-2 on every element"): each
+element must satisfy |gpu - oracle| <= 2e-2 + 2e-2 * |oracle|.
+"""
+import numpy as np
+import torch
+
+import oracle
+from paged_kv_cache_474_b200.workloads import Workload, bf16_bits
+
+ATOL = 2e-2
+RTOL = 2e-2
+
+
+def problem(wl: Workload) -> oracle.Problem:
+    """Whole workload as an oracle problem (host copies of every buffer)."""
+    return oracle.Problem(
+        bf16_bits(wl.q), bf16_bits(wl.k_cache), bf16_bits(wl.v_cache),
+        wl.block_tables.cpu().numpy(), wl.seq_lens.cpu().numpy(),
+        wl.query_lens.cpu().numpy(), wl.scale, wl.window,
+        None if wl.windows is None else wl.windows.cpu().numpy())
+
+
+def subproblem(wl: Workload, rows):
+    """Oracle problem holding only the given batch rows: their q rows, the
+    blocks their tables reach (gathered into a compact pool, tables
+    remapped), lengths and windows.  Returns (problem, row_map) where row_map
+    maps an original row to its index in the sub-problem."""
+    rows = sorted(set(int(r) for r in rows))
+    S = wl.seq_lens.cpu().tolist()
+    L = wl.query_lens.cpu().tolist()
+    W = wl.windows.cpu().tolist() if wl.windows is not None else None
+    bs = wl.block_size
+    tables = wl.block_tables.cpu()
+    qoff = np.concatenate([[0], np.cumsum(L)]).astype(np.int64)
+    phys = []
+    new_tables = []
+    for b in rows:
+        nb = (S[b] + bs - 1) // bs
+        ids = tables[b, :nb].tolist()
+        new_tables.append(list(range(len(phys), len(phys) + nb)))
+        phys.extend(ids)
+    mb = max(len(t) for t in new_tables)
+    tab = np.zeros((len(rows), mb), dtype=np.int32)
+    for j, t in enumerate(new_tables):
+        tab[j, :len(t)] = t
+    idx = torch.tensor(phys, dtype=torch.long, device=wl.k_cache.device)
+    kc = bf16_bits(wl.k_cache.index_select(0, idx))
+    vc = bf16_bits(wl.v_cache.index_select(0, idx))
+    qs = torch.cat([wl.q[qoff[b]:qoff[b + 1]] for b in rows])
+    pr = oracle.Problem(bf16_bits(qs), kc, vc, tab,
+                        np.array([S[b] for b in rows], dtype=np.int32),
+                        np.array([L[b] for b in rows], dtype=np.int32),
+                        wl.scale, wl.window,
+                        None if W is None else np.array([W[b] for b in rows], dtype=np.int32))
+    return pr, {b: j for j, b in enumerate(rows)}
+
+
+def token_offsets(wl: Workload):
+    L = wl.query_lens.cpu().tolist()
+    return np.concatenate([[0], np.cumsum(L)]).astype(np.int64)
+
+
+def assert_close(got, ref, what=""):
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite GPU output"
+    err = np.abs(got - ref)
+    bound = ATOL + RTOL * np.abs(ref)
+    bad = err > bound
+    if bad.any():
+        i = np.unravel_index(np.argmax(err - bound), err.shape)
+        raise AssertionError(
+            f"{what}: {int(bad.sum())} of {err.size} elements out of tolerance; "
+            f"worst at {i}: gpu={got[i]:.6f} oracle={ref[i]:.6f}")
+    return float(err.max())
+
+
+def check_full(wl: Workload, dst, what=""):
+    ref = oracle.decode(problem(wl))
+    return assert_close(dst.float().cpu().numpy(), ref, what)
+
+
+def sample_queries(wl: Workload, n: int, seed: int = 0, rows=None):
+    """n seeded (b, i, h) triples over rows with queryLen > 0 (or only `rows`)."""
+    g = np.random.default_rng(seed)
+    L = wl.query_lens.cpu().tolist()
+    cand = [b for b in (rows if rows is not None else range(wl.batch)) if L[b] > 0]
+    out = []
+    for _ in range(n):
+        b = int(g.choice(cand))
+        out.append((b, int(g.integers(0, L[b])), int(g.integers(0, wl.num_q_heads))))
+    return out
+
+
+def check_sampled(wl: Workload, dst, sel, what=""):
+    """Compares the outputs of the selected (b, i, h) with the oracle computed
+    one by one on a sub-problem holding only the rows involved."""
+    pr, rmap = subproblem(wl, [b for b, _, _ in sel])
+    ref = oracle.decode_select(pr, [(rmap[b], i, h) for b, i, h in sel])
+    qoff = token_offsets(wl)
+    d = dst.float().cpu().numpy()
+    got = np.stack([d[qoff[b] + i, h] for b, i, h in sel])
+    return assert_close(got, ref, what)

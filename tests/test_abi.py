@@ -1,0 +1,170 @@
+"""CPU checks of the C ABI: the library loads, exports every symbol the header
+declares, validates arguments on the host, and plans partitions the way the
+dispatcher promises.  No call here launches GPU work."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pagedattn.h")
+
+pa = pytest.importorskip("paged_kv_cache_474_b200")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("pa_decode", "pa_workspace_size", "pa_visible_ranges", "pa_last_error"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported_and_bound():
+    import ctypes
+    lib = ctypes.CDLL(pa.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert name in pa.SIGNATURES, name
+
+
+def test_version():
+    assert "sm_100a" in pa.pa_version()
+
+
+def base_params(**kw):
+    d = dict(batch=2, num_q_heads=4, num_kv_heads=2, head_dim=64, num_blocks=8,
+             max_blocks_per_seq=4, max_span_hint=50, max_query_len_hint=1)
+    d.update(kw)
+    return pa.make_params(**d)
+
+
+def call(p, bs=16, window=0, scale=0.125, ptrs=16):
+    return pa.pa_decode(ptrs, ptrs, ptrs, ptrs, ptrs, ptrs, ptrs, scale, window, bs, p, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(num_q_heads=5), pa.PA_ERR_ARG),
+    (dict(num_kv_heads=0), pa.PA_ERR_ARG),
+    (dict(head_dim=96), pa.PA_ERR_UNSUPPORTED),
+    (dict(head_dim=256), pa.PA_ERR_UNSUPPORTED),
+    (dict(batch=-1), pa.PA_ERR_ARG),
+    (dict(num_blocks=0), pa.PA_ERR_ARG),
+    (dict(max_span_hint=-3), pa.PA_ERR_ARG),
+    (dict(force_partitions=-1), pa.PA_ERR_ARG),
+    (dict(force_variant=7), pa.PA_ERR_ARG),
+])
+def test_invalid_params_are_rejected_on_the_host(kw, code):
+    assert call(base_params(**kw)) == code
+    assert pa.pa_last_error()
+
+
+@pytest.mark.parametrize("bs", [0, 8, 48, 2048])
+def test_unsupported_block_sizes(bs):
+    assert call(base_params(), bs=bs) == pa.PA_ERR_UNSUPPORTED
+
+
+def test_negative_window_null_and_misaligned_pointers():
+    assert call(base_params(), window=-1) == pa.PA_ERR_ARG
+    assert call(base_params(), ptrs=0) == pa.PA_ERR_ARG
+    assert call(base_params(), ptrs=24) == pa.PA_ERR_ARG
+    assert call(base_params(), scale=float("nan")) == pa.PA_ERR_ARG
+
+
+def test_empty_batch_is_a_no_op():
+    assert call(base_params(batch=0)) == pa.PA_OK
+    assert pa.pa_last_error() == ""
+
+
+def test_extents_follow_the_window_rule():
+    # gllm page "Verification" batch: a 5-token chunk over 300 and a decode row over 40
+    assert pa.pa_extents_host([300, 40], [5, 1], 16) == (20, 5)
+    assert pa.pa_extents_host([300, 40], [5, 1], 0) == (300, 5)
+    assert pa.pa_extents_host([300, 40], [5, 1], 4096) == (300, 5)
+    assert pa.pa_extents_host([300, 40], [0, 1], 16) == (16, 1)
+    assert pa.pa_extents_host([7, 9], [3, 1], windows=[2, 0]) == (9, 3)
+    assert pa.pa_extents_host([7, 9], [3, 1], windows=[2, 5]) == (5, 3)
+    with pytest.raises(pa.PagedAttnError):
+        pa.pa_extents_host([3], [4], 0)
+
+
+def test_extents_agree_with_oracle_ranges():
+    rng = np.random.default_rng(0)
+    for _ in range(50):
+        B = int(rng.integers(1, 20))
+        S = rng.integers(1, 5000, B)
+        L = np.minimum(S, rng.integers(0, 6, B))
+        W = rng.choice([0, 1, 7, 64, 4096], B)
+        lo, hi = oracle.visible_ranges(S, L, windows=W)
+        span, qlen = pa.pa_extents_host(S, L, windows=W)
+        qoff = np.concatenate([[0], np.cumsum(L)])
+        want = max([int(S[b] - lo[qoff[b]]) for b in range(B) if L[b] > 0] or [0])
+        assert span == want and qlen == int(L.max())
+
+
+def plan(**kw):
+    bs = kw.pop("bs", 16)
+    sms = kw.pop("sms", 148)
+    occ = kw.pop("occ", 2)
+    rc, info = pa.pa_plan(base_params(**kw), bs, sms, occ)
+    assert rc == pa.PA_OK, pa.pa_last_error()
+    return info
+
+
+def test_plan_long_single_group_fills_one_wave():
+    # B=1, H_kv=1, S=131072: partitions sized so one wave covers every SM slot
+    info = plan(batch=1, num_q_heads=8, num_kv_heads=1, head_dim=128, num_blocks=8193,
+                max_blocks_per_seq=8192, max_span_hint=131072)
+    assert info.partition_tokens % 64 == 0
+    assert info.max_partitions * info.partition_tokens >= 131072 + 63
+    assert 148 * 2 * 0.9 <= info.max_partitions <= 148 * 2
+    assert not info.one_shot and info.workspace_bytes > 0
+    assert info.grid_x == info.max_partitions and info.grid_y == 1 and info.grid_z == 1
+
+
+def test_plan_uses_the_windowed_span_not_the_context():
+    wide = plan(batch=16, num_q_heads=32, num_kv_heads=8, head_dim=128, num_blocks=30000,
+                max_blocks_per_seq=2048, max_span_hint=32768, max_query_len_hint=5)
+    windowed = plan(batch=16, num_q_heads=32, num_kv_heads=8, head_dim=128, num_blocks=30000,
+                    max_blocks_per_seq=2048, max_span_hint=4100, max_query_len_hint=5)
+    assert windowed.max_partitions * windowed.partition_tokens < 8192
+    assert wide.max_partitions * wide.partition_tokens >= 32768
+
+
+def test_plan_one_shot_for_short_spans():
+    info = plan(max_span_hint=50)
+    assert info.one_shot and info.max_partitions == 1 and info.workspace_bytes == 0
+
+
+def test_plan_forced_partitions_and_workspace_formula():
+    info = plan(batch=3, num_q_heads=8, num_kv_heads=2, head_dim=128, num_blocks=400,
+                max_blocks_per_seq=320, max_span_hint=5000, max_query_len_hint=3,
+                force_partitions=7)
+    assert info.partition_tokens == 768 and info.max_partitions == 7
+    rows = 4 * 3
+    partials = 3 * 2 * 7 * rows
+    align = lambda x: (x + 255) // 256 * 256
+    assert info.max_rows == rows
+    assert info.workspace_bytes == align(partials * 4) + align(partials * 128 * 4)
+
+
+def test_plan_row_slabs_for_many_rows():
+    info = plan(batch=4, num_q_heads=64, num_kv_heads=8, head_dim=128, num_blocks=400,
+                max_blocks_per_seq=64, bs=1024, max_span_hint=65536, max_query_len_hint=4)
+    assert info.max_rows == 32 and info.slab_rows == 32 and info.grid_y == 8
+    big = plan(batch=2, num_q_heads=64, num_kv_heads=4, head_dim=128, num_blocks=400,
+               max_blocks_per_seq=64, bs=1024, max_span_hint=65536, max_query_len_hint=5)
+    assert big.max_rows == 80 and big.grid_y == 4 * 3
+
+
+def test_plan_caps_partition_at_the_table_cache():
+    info = plan(batch=1, num_q_heads=1, num_kv_heads=1, head_dim=64, num_blocks=70000,
+                max_blocks_per_seq=65536, max_span_hint=1 << 20, sms=1, occ=1)
+    assert info.partition_tokens <= (1024 - 2) * 16

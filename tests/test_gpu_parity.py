@@ -1,0 +1,292 @@
+"""GPU parity: pa_decode (through the C ABI) against the float64 oracle.
+
+Small workloads are compared element by element; the five named workloads
+at full size are compared on seeded samples the oracle computes one by one,
+in the same launch configuration the bench times (host hints, workspace,
+dispatcher's partitioning).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests.parity_helpers import (assert_close, check_full, check_sampled,
+                                  problem, sample_queries, token_offsets)
+
+pytestmark = pytest.mark.gpu
+
+pa = pytest.importorskip("paged_kv_cache_474_b200")
+from paged_kv_cache_474_b200.workloads import (config_lengths, config_workload,  # noqa: E402
+                                               make_workload)
+
+
+@pytest.fixture(autouse=True)
+def _device_status_clean(cuda_device):
+    pa.pa_device_status(clear=True)
+    yield
+    assert pa.pa_device_status(clear=True) == 0
+
+
+def dev(wl):
+    return wl.to("cuda:0")
+
+
+# ----------------------------------------------------------- small, full
+@pytest.mark.parametrize("window", [0, 8])
+@pytest.mark.parametrize("parts", [0, 1, 2, 3])
+def test_tiny_workload(window, parts):
+    wl = config_workload(1, window=window)
+    out = pa.decode(dev(wl), force_partitions=parts)
+    check_full(wl, out, f"tiny w={window} parts={parts}")
+
+
+def scaled(cfg, seed=1):
+    """The named workloads' shapes at lengths the oracle finishes in seconds,
+    still spanning several stages, partitions and a ragged tail."""
+    g = np.random.default_rng(seed)
+    if cfg == 2:
+        s = g.integers(100, 1500, 6).tolist()
+        return make_workload(seq_lens=s, query_lens=[1] * 6, num_q_heads=32,
+                             num_kv_heads=8, head_dim=128, block_size=16, seed=seed)
+    if cfg == 3:
+        s = g.integers(200, 2500, 7).tolist() + [300]
+        return make_workload(seq_lens=s, query_lens=[1, 1, 1, 1, 2, 3, 4, 5],
+                             num_q_heads=32, num_kv_heads=8, head_dim=128,
+                             block_size=16, window=333, seed=seed)
+    if cfg == 4:
+        return make_workload(seq_lens=[9001], query_lens=[1], num_q_heads=8,
+                             num_kv_heads=1, head_dim=128, block_size=16, seed=seed)
+    if cfg == 5:
+        s = g.integers(1100, 4200, 6).tolist()
+        l = g.integers(1, 5, 6).tolist()
+        return make_workload(seq_lens=s, query_lens=l, num_q_heads=64,
+                             num_kv_heads=8, head_dim=128, block_size=1024,
+                             windows=[700 if b % 2 == 0 else 0 for b in range(6)],
+                             seed=seed)
+    raise ValueError(cfg)
+
+
+@pytest.mark.parametrize("cfg", [2, 3, 4, 5])
+@pytest.mark.parametrize("parts", [0, 1, 5])
+def test_scaled_named_workloads(cfg, parts):
+    wl = scaled(cfg)
+    out = pa.decode(dev(wl), force_partitions=parts)
+    check_full(wl, out, f"scaled cfg{cfg} parts={parts}")
+
+
+@pytest.mark.parametrize("parts", [1, 2, 3, 7, 64, 200])
+def test_split_k_invariance(parts):
+    wl = make_workload(seq_lens=[5000, 3333, 77], query_lens=[1, 3, 2], num_q_heads=8,
+                       num_kv_heads=2, head_dim=128, block_size=16, window=0, seed=7)
+    d = dev(wl)
+    out = pa.decode(d, force_partitions=parts)
+    check_full(wl, out, f"parts={parts}")
+    base = pa.decode(d, force_partitions=1).float()
+    assert torch.max(torch.abs(out.float() - base)).item() < 2e-2
+
+
+@pytest.mark.parametrize("head_dim", [64, 128])
+@pytest.mark.parametrize("block_size", [16, 32, 64, 256, 1024])
+def test_head_dims_and_block_sizes(head_dim, block_size):
+    wl = make_workload(seq_lens=[1, 17, 64, 65, 1500, 2049], query_lens=[1, 1, 2, 1, 4, 1],
+                       num_q_heads=8, num_kv_heads=4, head_dim=head_dim,
+                       block_size=block_size, window=0, seed=head_dim + block_size)
+    out = pa.decode(dev(wl))
+    check_full(wl, out, f"D={head_dim} BS={block_size}")
+
+
+@pytest.mark.parametrize("window", [1, 2, 5, 16, 100, 4096])
+def test_gllm_window_batch(window):
+    # gllm PR #116 "Verification": a 5-token prefill chunk over a 300-token
+    # context plus a decode row over 40, windows 16, 100 and 4096 (and the
+    # CPU test's small windows), here with GQA.
+    wl = make_workload(seq_lens=[300, 40], query_lens=[5, 1], num_q_heads=8,
+                       num_kv_heads=2, head_dim=64, block_size=16, window=window,
+                       seed=window)
+    out = pa.decode(dev(wl))
+    check_full(wl, out, f"window={window}")
+
+
+def test_window_one_returns_own_value():
+    wl = make_workload(seq_lens=[70, 3, 1000], query_lens=[3, 1, 2], num_q_heads=4,
+                       num_kv_heads=2, head_dim=128, block_size=16, window=1, seed=3)
+    out = pa.decode(dev(wl)).cpu()
+    qoff = token_offsets(wl)
+    for b, (S, L) in enumerate(zip(wl.seq_lens.tolist(), wl.query_lens.tolist())):
+        for i in range(L):
+            p = S - L + i
+            phys = int(wl.block_tables[b, p // 16])
+            for h in range(4):
+                assert torch.equal(out[qoff[b] + i, h], wl.v_cache[phys, h // 2, p % 16])
+
+
+def test_window_at_or_beyond_context_equals_unlimited():
+    kw = dict(seq_lens=[500, 123, 2000], query_lens=[1, 2, 1], num_q_heads=8,
+              num_kv_heads=1, head_dim=128, block_size=16, seed=4)
+    a = pa.decode(dev(make_workload(window=0, **kw)))
+    b = pa.decode(dev(make_workload(window=2000, **kw)))
+    c = pa.decode(dev(make_workload(window=10 ** 6, **kw)))
+    assert torch.equal(a, b) and torch.equal(a, c)
+
+
+def test_rows_without_queries_and_empty_batch():
+    wl = make_workload(seq_lens=[50, 900, 10, 333], query_lens=[0, 2, 0, 1], num_q_heads=4,
+                       num_kv_heads=4, head_dim=64, block_size=16, seed=5)
+    out = pa.decode(dev(wl))
+    check_full(wl, out, "zero-length rows")
+    empty = make_workload(seq_lens=[], query_lens=[], num_q_heads=4, num_kv_heads=4,
+                          head_dim=64, block_size=16, seed=5)
+    p = pa.params_for(empty)
+    rc = pa.pa_decode(16, 16, 16, 16, 16, 16, 16, 1.0, 0, 16, p, None)
+    assert rc == pa.PA_OK
+
+
+def test_garbage_outside_spans_is_never_read():
+    # Slots past each row's last token, the spare block and unused table
+    # entries hold NaN / out-of-range values; outputs must not see them.
+    wl = make_workload(seq_lens=[37, 50, 1], query_lens=[1, 3, 1], num_q_heads=4,
+                       num_kv_heads=2, head_dim=128, block_size=16, window=0, seed=9,
+                       spare_blocks=2, extra_table_cols=3)
+    ref = oracle.decode(problem(wl))
+    for b, S in enumerate(wl.seq_lens.tolist()):
+        nb = (S + 15) // 16
+        last = int(wl.block_tables[b, nb - 1])
+        wl.k_cache[last, :, S - (nb - 1) * 16:] = float("nan")
+        wl.v_cache[last, :, S - (nb - 1) * 16:] = float("nan")
+        wl.block_tables[b, nb:] = 10 ** 6
+    used = set(wl.block_tables[wl.block_tables < wl.num_blocks].tolist())
+    for blk in range(wl.num_blocks):
+        if blk not in used:
+            wl.k_cache[blk] = float("nan")
+            wl.v_cache[blk] = float("nan")
+    out = pa.decode(dev(wl))
+    assert_close(out.float().cpu().numpy(), ref, "garbage outside spans")
+
+
+def test_no_hints_path_matches_hinted():
+    wl = scaled(3)
+    d = dev(wl)
+    a = pa.decode(d, hints=True)
+    b = pa.decode(d, hints=False)
+    assert torch.equal(a, b)
+
+
+def test_visible_ranges_match_oracle_exactly():
+    cases = [config_lengths(c) for c in (1, 2, 3, 4, 5)]
+    cases += [([300, 40], [5, 1], w, None) for w in (0, 1, 2, 5, 16, 100, 4096)]
+    cases += [([7, 1, 9, 2500, 33] * 300, [3, 1, 0, 5, 2] * 300, 0, [2, 0, 4, 333, 1] * 300)]
+    for s, l, w, ws in cases:
+        S = torch.tensor(s, dtype=torch.int32, device="cuda:0")
+        L = torch.tensor(l, dtype=torch.int32, device="cuda:0")
+        W = None if ws is None else torch.tensor(ws, dtype=torch.int32, device="cuda:0")
+        lo, hi = pa.visible_ranges(S, L, w, W)
+        rlo, rhi = oracle.visible_ranges(s, l, w, ws)
+        assert np.array_equal(lo.cpu().numpy(), rlo)
+        assert np.array_equal(hi.cpu().numpy(), rhi)
+
+
+def test_host_entry_point_matches_device_path():
+    wl = scaled(5)
+    d = dev(wl)
+    ref = pa.decode(d)
+    s, l, w = wl.host_lists()
+    p = pa.make_params(batch=wl.batch, num_q_heads=wl.num_q_heads,
+                       num_kv_heads=wl.num_kv_heads, head_dim=wl.head_dim,
+                       num_blocks=wl.num_blocks, max_blocks_per_seq=wl.max_blocks_per_seq)
+    S = wl.seq_lens.numpy().copy()
+    L = wl.query_lens.numpy().copy()
+    W = wl.windows.numpy().copy()
+    p.windows = W.ctypes.data
+    n = pa.pa_host_workspace_size(p, wl.block_size, wl.window, S.ctypes.data, L.ctypes.data)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda:0")
+    p.workspace, p.workspace_bytes = ws.data_ptr(), n
+    q_host = wl.q.contiguous().pin_memory()
+    out_host = torch.empty_like(wl.q).pin_memory()
+    bt = wl.block_tables.contiguous().numpy()
+    rc = pa.pa_decode_host(out_host.data_ptr(), q_host.data_ptr(), d.k_cache.data_ptr(),
+                           d.v_cache.data_ptr(), bt.ctypes.data, S.ctypes.data, L.ctypes.data,
+                           wl.scale, wl.window, wl.block_size, p,
+                           pa._stream_handle())
+    assert rc == pa.PA_OK, pa.pa_last_error()
+    assert torch.equal(out_host, ref.cpu())
+
+
+# ---------------------------------------------------- full size, sampled
+@pytest.mark.parametrize("cfg", [2, 3, 4, 5])
+def test_named_workload_full_size_sampled(cfg):
+    wl = config_workload(cfg, device="cuda:0")
+    out = pa.decode(wl)
+    torch.cuda.synchronize()
+    n = 48
+    sel = sample_queries(wl, n, seed=cfg)
+    if cfg in (3, 5):   # make sure every kind of row is sampled
+        L = wl.query_lens.cpu().tolist()
+        kinds = {}
+        for b, l in enumerate(L):
+            kinds.setdefault((l, None if wl.windows is None else int(wl.windows[b])), b)
+        for b in kinds.values():
+            sel += [(b, L[b] - 1, 0), (b, 0, wl.num_q_heads - 1)]
+    if cfg == 5:       # keep the gathered sub-problem small: few distinct rows
+        rows = sorted({b for b, _, _ in sel})[:6]
+        sel = [t for t in sel if t[0] in rows]
+    check_sampled(wl, out, sel, f"cfg{cfg} full size")
+
+
+# ------------------------------------------------------------ error paths
+def test_small_workspace_is_rejected():
+    wl = dev(scaled(4))
+    p = pa.params_for(wl)
+    need = pa.pa_workspace_size(p, wl.block_size)
+    assert need > 0
+    ws = torch.empty(need - 256, dtype=torch.uint8, device="cuda:0")
+    p.workspace, p.workspace_bytes = ws.data_ptr(), ws.numel()
+    out = torch.empty_like(wl.q)
+    rc = pa.pa_decode(out.data_ptr(), wl.q.data_ptr(), wl.k_cache.data_ptr(),
+                      wl.v_cache.data_ptr(), wl.block_tables.data_ptr(),
+                      wl.seq_lens.data_ptr(), wl.query_lens.data_ptr(), wl.scale,
+                      wl.window, wl.block_size, p, pa._stream_handle())
+    assert rc == pa.PA_ERR_WORKSPACE
+
+
+def _raw_decode(wl, p, out):
+    return pa.pa_decode(out.data_ptr(), wl.q.data_ptr(), wl.k_cache.data_ptr(),
+                        wl.v_cache.data_ptr(), wl.block_tables.data_ptr(),
+                        wl.seq_lens.data_ptr(), wl.query_lens.data_ptr(), wl.scale,
+                        wl.window, wl.block_size, p, pa._stream_handle())
+
+
+def test_device_detects_rows_beyond_hints_and_bad_blocks():
+    wl = dev(make_workload(seq_lens=[900, 40], query_lens=[1, 1], num_q_heads=4,
+                           num_kv_heads=2, head_dim=64, block_size=16, seed=2))
+    # span hint smaller than the real span: the long row is skipped and flagged
+    p = pa.params_for(wl)
+    p.max_span_hint = 100
+    ws = pa.alloc_workspace(p, 16)
+    if ws is not None:
+        p.workspace, p.workspace_bytes = ws.data_ptr(), ws.numel()
+    out = torch.zeros_like(wl.q)
+    assert _raw_decode(wl, p, out) == pa.PA_OK
+    assert pa.pa_device_status(clear=True) & pa.PA_DEV_HINT
+    # a block-table entry outside the pool is flagged, not dereferenced
+    bad = wl.block_tables.clone()
+    bad[1, 0] = wl.num_blocks + 5
+    wl2 = type(wl)(**{**wl.__dict__, "block_tables": bad})
+    p = pa.params_for(wl2)
+    ws = pa.alloc_workspace(p, 16)
+    if ws is not None:
+        p.workspace, p.workspace_bytes = ws.data_ptr(), ws.numel()
+    assert _raw_decode(wl2, p, out) == pa.PA_OK
+    assert pa.pa_device_status(clear=True) & pa.PA_DEV_BAD_BLOCK
+    # a row whose queryLen exceeds its seqLen is flagged when hints skip the host check
+    lens = torch.tensor([900, 2], dtype=torch.int32, device="cuda:0")
+    ql = torch.tensor([1, 3], dtype=torch.int32, device="cuda:0")
+    wl3 = type(wl)(**{**wl.__dict__, "query_lens": ql, "seq_lens": lens,
+                      "q": torch.zeros(4, 4, 64, dtype=torch.bfloat16, device="cuda:0")})
+    p = pa.params_for(wl, hints=False)
+    p.max_span_hint, p.max_query_len_hint = 900, 3
+    ws = pa.alloc_workspace(p, 16)
+    if ws is not None:
+        p.workspace, p.workspace_bytes = ws.data_ptr(), ws.numel()
+    out3 = torch.zeros(4, 4, 64, dtype=torch.bfloat16, device="cuda:0")
+    assert _raw_decode(wl3, p, out3) == pa.PA_OK
+    assert pa.pa_device_status(clear=True) & pa.PA_DEV_BAD_ROW
