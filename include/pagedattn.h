@@ -67,7 +67,8 @@ extern "C" {
 
 /* Kernel variants (pa_params.force_variant, pa_plan_info.variant). */
 #define PA_VARIANT_AUTO 0
-#define PA_VARIANT_FMA 1      /* CUDA-core FMA scores and PV (few rows per kv head) */
+#define PA_VARIANT_FMA 1      /* CUDA-core FMA scores and PV (group x queryLen <= 4 rows) */
+#define PA_VARIANT_MMA 2      /* tensor-core m16n8k16 tiles with TMA-swizzled staging (dense rows) */
 
 typedef struct pa_params {
     int batch;               /* rows */
@@ -88,6 +89,10 @@ typedef struct pa_params {
     size_t workspace_bytes;
     int force_variant;       /* PA_VARIANT_AUTO, or a PA_VARIANT_* for tests and A/B runs */
     int force_partitions;    /* 0 = dispatcher's choice; n > 0 cuts the longest span into ~n partitions */
+    /* Optional instrumentation: NULL, or a host array of two cudaEvent_t that
+     * pa_decode records on the stream immediately before and after the
+     * partition kernel (the reduce, if any, runs after the second). */
+    void *const *profile_events;
 } pa_params;
 
 /* What the dispatcher chose for a call (pa_plan). */

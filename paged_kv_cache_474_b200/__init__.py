@@ -31,6 +31,7 @@ PA_DEV_HINT = 8
 
 PA_VARIANT_AUTO = 0
 PA_VARIANT_FMA = 1
+PA_VARIANT_MMA = 2
 
 
 class pa_params(ctypes.Structure):
@@ -48,6 +49,7 @@ class pa_params(ctypes.Structure):
         ("workspace_bytes", ctypes.c_size_t),
         ("force_variant", ctypes.c_int),
         ("force_partitions", ctypes.c_int),
+        ("profile_events", ctypes.c_void_p),
     ]
 
 

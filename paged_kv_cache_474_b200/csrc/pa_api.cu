@@ -20,6 +20,9 @@
 #include <string>
 #include <vector>
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "../../include/pagedattn.h"
 #include "pa_kernels.cuh"
 #include "pa_span.h"
@@ -98,7 +101,8 @@ int check_params(const pa_params* p, int bs) {
   if (p->max_span_hint < 0 || p->max_query_len_hint < 0)
     return fail(PA_ERR_ARG, "hints must be >= 0");
   if (p->force_partitions < 0) return fail(PA_ERR_ARG, "force_partitions must be >= 0");
-  if (p->force_variant != PA_VARIANT_AUTO && p->force_variant != PA_VARIANT_FMA)
+  if (p->force_variant != PA_VARIANT_AUTO && p->force_variant != PA_VARIANT_FMA &&
+      p->force_variant != PA_VARIANT_MMA)
     return fail(PA_ERR_ARG, "unknown force_variant %d", p->force_variant);
   return PA_OK;
 }
@@ -120,8 +124,18 @@ int make_plan(const pa_params* p, int bs, int span, int qlen, int num_sms, int c
   if ((long long)G * qlen > 4096)
     return fail(PA_ERR_UNSUPPORTED, "rows per kv head %lld exceed 4096", (long long)G * qlen);
   const int rmax = G * qlen;
-  const int ncw = rmax <= 16 ? 4 : 8;
-  const int slab_rows = 4 * ncw;
+  // Variant: tensor-core tiles once the rows of a (row, kv head) unit fill a
+  // real tile (8 or more), CUDA-core FMA below that.  The tensor-core path
+  // addresses cache rows through a TMA map with 32-bit row coordinates.
+  const bool rows_fit_tma =
+      (long long)p->num_blocks * p->num_kv_heads * bs <= (long long)INT32_MAX;
+  int variant = p->force_variant;
+  if (variant == PA_VARIANT_AUTO) variant = (rmax > 4 && rows_fit_tma) ? PA_VARIANT_MMA : PA_VARIANT_FMA;
+  if (variant == PA_VARIANT_MMA && !rows_fit_tma)
+    return fail(PA_ERR_UNSUPPORTED, "KV pool rows exceed the tensor map's 32-bit coordinates");
+  const bool mma = variant == PA_VARIANT_MMA;
+  const int ncw = mma ? 4 : (rmax <= 16 ? 4 : 8);
+  const int slab_rows = mma ? 16 * ncw : 4 * ncw;
   const int nslab = (int)cdiv(rmax, slab_rows);
   pl.shape.head_dim = p->head_dim;
   pl.shape.consumer_warps = ncw;
@@ -129,13 +143,17 @@ int make_plan(const pa_params* p, int bs, int span, int qlen, int num_sms, int c
 
   // Partition-size cap: the CTA caches its slice of the block table in smem.
   const int cap = std::max(TS, ((pa::kMaxTableCache - 2) * bs) / TS * TS);
-  const size_t smem_max = pa::fma_smem_bytes(p->head_dim, pl.shape.stages, cap, bs);
+  auto smem_for = [&](int ptok) {
+    return mma ? pa::mma_smem_bytes(p->head_dim, pl.shape.stages, ptok, bs)
+               : pa::fma_smem_bytes(p->head_dim, pl.shape.stages, ptok, bs);
+  };
   if (num_sms <= 0) {
     int rc = current_sms(&num_sms);
     if (rc) return rc;
   }
   if (ctas_per_sm <= 0) {
-    ctas_per_sm = pa::occupancy_partition_fma(pl.shape, smem_max);
+    ctas_per_sm = mma ? pa::occupancy_partition_mma(pl.shape, smem_for(cap))
+                      : pa::occupancy_partition_fma(pl.shape, smem_for(cap));
     if (ctas_per_sm <= 0)
       return fail(PA_ERR_CUDA, "occupancy query failed: %s", cudaGetErrorString(cudaGetLastError()));
   }
@@ -156,7 +174,7 @@ int make_plan(const pa_params* p, int bs, int span, int qlen, int num_sms, int c
   if (max_parts > (1LL << 30)) return fail(PA_ERR_UNSUPPORTED, "too many partitions");
 
   pa_plan_info& in = pl.info;
-  in.variant = PA_VARIANT_FMA;
+  in.variant = variant;
   in.partition_tokens = (int)ptok;
   in.max_partitions = (int)max_parts;
   in.one_shot = max_parts == 1;
@@ -168,7 +186,7 @@ int make_plan(const pa_params* p, int bs, int span, int qlen, int num_sms, int c
   in.grid_y = p->num_kv_heads * nslab;
   in.grid_z = p->batch;
   in.block_threads = 32 * (ncw + 1);
-  in.smem_bytes = pa::fma_smem_bytes(p->head_dim, pl.shape.stages, (int)ptok, bs);
+  in.smem_bytes = smem_for((int)ptok);
   in.num_sms = num_sms;
   in.ctas_per_sm = ctas_per_sm;
   if (!in.one_shot) {
@@ -178,6 +196,65 @@ int make_plan(const pa_params* p, int bs, int span, int qlen, int num_sms, int c
     in.workspace_bytes = pl.lse_bytes + pl.o_bytes;
   }
   *out = pl;
+  return PA_OK;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// 2-D map of a KV cache viewed as [num_blocks * H_kv * BS rows][head_dim]
+// bf16: boxes of 64 elements (128 bytes, the swizzle span) x box_rows rows,
+// 128-byte swizzle.  Encodings are cached per (base, rows, head_dim, box_rows).
+int kv_tensor_map(CUtensorMap* out, const void* base, long long rows, int head_dim, int box_rows) {
+  struct Entry {
+    const void* base;
+    long long rows;
+    int d, br;
+    CUtensorMap map;
+  };
+  static std::mutex mu;
+  static std::vector<Entry> cache;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Entry& e : cache)
+      if (e.base == base && e.rows == rows && e.d == head_dim && e.br == box_rows) {
+        *out = e.map;
+        return PA_OK;
+      }
+  }
+  auto fn = encode_fn();
+  if (!fn) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  const cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
+  const cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1u, 1u};
+  Entry e;
+  e.base = base;
+  e.rows = rows;
+  e.d = head_dim;
+  e.br = box_rows;
+  const CUresult r = fn(&e.map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache.size() >= 16) cache.erase(cache.begin());
+  cache.push_back(e);
+  *out = e.map;
   return PA_OK;
 }
 
@@ -263,7 +340,26 @@ int decode_impl(void* dst, const void* q, const void* kCache, const void* vCache
   a.num_slabs = in.grid_y / p->num_kv_heads;
 
   const dim3 grid(in.grid_x, in.grid_y, in.grid_z);
-  cudaError_t e = pa::launch_partition_fma(a, pl.shape, grid, in.smem_bytes, stream);
+  cudaEvent_t ev0 = nullptr, ev1 = nullptr;
+  if (p->profile_events) {
+    ev0 = static_cast<cudaEvent_t>(p->profile_events[0]);
+    ev1 = static_cast<cudaEvent_t>(p->profile_events[1]);
+  }
+  cudaError_t e = ev0 ? cudaEventRecord(ev0, stream) : cudaSuccess;
+  if (e == cudaSuccess) {
+    if (in.variant == PA_VARIANT_MMA) {
+      CUtensorMap tk, tv;
+      const long long rows = (long long)p->num_blocks * p->num_kv_heads * bs;
+      const int br = std::min(bs, TS);
+      rc = kv_tensor_map(&tk, kCache, rows, p->head_dim, br);
+      if (!rc) rc = kv_tensor_map(&tv, vCache, rows, p->head_dim, br);
+      if (rc) return rc;
+      e = pa::launch_partition_mma(a, pl.shape, tk, tv, grid, in.smem_bytes, stream);
+    } else {
+      e = pa::launch_partition_fma(a, pl.shape, grid, in.smem_bytes, stream);
+    }
+  }
+  if (e == cudaSuccess && ev1) e = cudaEventRecord(ev1, stream);
   if (e != cudaSuccess) return fail(PA_ERR_CUDA, "partition kernel launch: %s", cudaGetErrorString(e));
   if (!in.one_shot) {
     e = pa::launch_reduce(a, stream);

@@ -14,6 +14,8 @@
 // staged K/V row once for every query row of the GQA group.
 #include <climits>
 
+#include <cuda.h>
+
 #include "pa_device.cuh"
 #include "pa_kernels.cuh"
 
@@ -387,6 +389,357 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
 }
 
 // ---------------------------------------------------------------------------
+// Partition kernel, tensor-core variant (rows = GQA group x query tokens form
+// a dense tile: group x queryLen >= 8).
+//
+// Staging: the copy warp loads whole KV boxes (one block for 16/32/64-token
+// blocks, a 64-token slice of larger blocks) with 2-D tiled TMA copies and
+// the 128-byte swizzle, so each stage holds K then V as [D/64][64 tokens]
+// [128 B] with 16-byte chunk c of token t stored at chunk c ^ (t & 7): every
+// ldmatrix below reads 8 distinct bank groups.  Compute: each compute warp
+// owns a 16-row M tile (rows past the real ones are padding) and a slice of
+// the stage's 16-token chunks; S = Q K^T and O += P V run as m16n8k16 bf16
+// MMAs with fp32 accumulation, P staying in registers between the two.
+// Tokens a box brings in from outside the row's visible union (the head of
+// the first block, the tail of the last) get score -inf and their V lanes
+// are zeroed in registers, so uninitialised cache slots never reach O.
+// ---------------------------------------------------------------------------
+template <int D>
+struct MmaTraits {
+  static constexpr int HALVES = D / 64;
+  static constexpr int HALF_BYTES = TS * 128;
+  static constexpr int KV_BYTES = HALVES * HALF_BYTES;
+  static constexpr int STAGE_BYTES = 2 * KV_BYTES;
+  static constexpr int KSTEPS = D / 16;
+  static constexpr int NT = D / 8;  // 8-wide output column tiles
+};
+
+template <int D, int NCW>
+struct MmaCombine {
+  static constexpr int ACC_FLOATS = NCW * 16 * D;
+  static constexpr int L_FLOATS = NCW * 16;
+  static constexpr int M_FLOATS = NCW * 16;
+  static constexpr int BYTES = (ACC_FLOATS + L_FLOATS + M_FLOATS) * 4;
+};
+
+// Byte offset of 16-byte chunk `chunk` (0 .. D/8-1) of stage token row t.
+__device__ __forceinline__ uint32_t swz(int t, int chunk) {
+  return (uint32_t)((chunk >> 3) * (TS * 128) + t * 128 + (((chunk & 7) ^ (t & 7)) << 4));
+}
+
+template <int D, int NCW, int NSTAGE>
+__global__ void __launch_bounds__(32 * (NCW + 1), 1)
+    pa_partition_mma_kernel(const __grid_constant__ DecodeArgs a,
+                            const __grid_constant__ CUtensorMap tmk,
+                            const __grid_constant__ CUtensorMap tmv) {
+  using T = MmaTraits<D>;
+  using C = MmaCombine<D, NCW>;
+  static_assert(C::BYTES <= NSTAGE * T::STAGE_BYTES, "combine area must fit in the ring");
+
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  // 128-byte-swizzled TMA destinations must sit on 1024-byte boundaries.
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NSTAGE * T::STAGE_BYTES);
+  int* bt_s = reinterpret_cast<int*>(bars + 2 * NSTAGE);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int b = blockIdx.z;
+  const int kvh = blockIdx.y % a.num_kv_heads;
+  const int slab = blockIdx.y / a.num_kv_heads;
+  const int part = blockIdx.x;
+
+  const int S = a.seq_lens[b];
+  const int L = a.query_lens[b];
+  const int w = a.windows ? a.windows[b] : a.window;
+  if (L <= 0) return;
+  const bool lead = (part == 0 && slab == 0 && kvh == 0 && threadIdx.x == 0);
+  if (L > S || w < 0 || S > a.max_blocks_per_seq * a.block_size) {
+    if (lead) atomicOr(&g_pa_status, PA_DEV_BAD_ROW);
+    return;
+  }
+  const int R = a.group * L;
+  const int ulo = union_lo(S, L, w);
+  const int A = ulo & ~(TS - 1);
+  const int nparts = (S - A + a.part_tokens - 1) / a.part_tokens;
+  if (R > a.max_rows || nparts > a.max_parts) {
+    if (lead) atomicOr(&g_pa_status, PA_DEV_HINT);
+    return;
+  }
+  const int row0 = slab * a.slab_rows;
+  if (row0 >= R || part >= nparts) return;
+  const int Rs = min(a.slab_rows, R - row0);
+  const int p0 = A + part * a.part_tokens;
+  const int p1 = min(S, p0 + a.part_tokens);
+  const int nst = (p1 - p0 + TS - 1) / TS;
+  const int jb0 = p0 >> a.block_shift;
+  const int nbt = ((p1 - 1) >> a.block_shift) - jb0 + 1;
+
+  for (int i = threadIdx.x; i < nbt; i += blockDim.x) {
+    int phys = a.block_tables[(size_t)b * a.max_blocks_per_seq + jb0 + i];
+    if (phys < 0 || phys >= a.num_blocks) {
+      atomicOr(&g_pa_status, PA_DEV_BAD_BLOCK);
+      phys = -1;
+    }
+    bt_s[i] = phys;
+  }
+  if (threadIdx.x == 0) {
+    prefetch_tensormap(&tmk);
+    prefetch_tensormap(&tmv);
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(smem_u32(&bars[s]), 1);
+      mbar_init(smem_u32(&bars[NSTAGE + s]), NCW);
+    }
+    fence_mbar_init();
+  }
+  const int qoff = row_token_offset(a.query_lens, b, lane);
+  __syncthreads();
+
+  float* comb_acc = reinterpret_cast<float*>(smem);
+  float* comb_l = comb_acc + C::ACC_FLOATS;
+  float* comb_m = comb_l + C::L_FLOATS;
+  const int NMT = (Rs + 15) >> 4;  // 16-row M tiles in this slab
+
+  if (warp == 0) {
+    // ------------------------------ copy warp ------------------------------
+    const int BR = min(a.block_size, TS);  // rows per box
+    const int nbox = TS / BR;
+    const int nitem = nbox * 2 * T::HALVES;  // (box, K/V, half) per lane
+    const uint32_t box_bytes = (uint32_t)BR * 128u;
+    int issued = 0;
+    for (int k = 0; k < nst; ++k) {
+      const int s = k % NSTAGE;
+      if (k >= NSTAGE) {
+        bool got = true;
+        if (lane == 0) got = mbar_wait(smem_u32(&bars[NSTAGE + s]), ((k / NSTAGE) - 1) & 1);
+        if (!__shfl_sync(FULL, got, 0)) break;
+      }
+      const int c0 = p0 + k * TS;
+      const int ta = max(c0, ulo), te = min(c0 + TS, p1);
+      bool mine = false;
+      uint32_t dst = 0;
+      int x = 0, y = 0, isv = 0;
+      if (lane < nitem) {
+        const int j = lane / (2 * T::HALVES);
+        const int rem = lane - j * (2 * T::HALVES);
+        isv = rem / T::HALVES;
+        const int h = rem - isv * T::HALVES;
+        const int bt0 = c0 + j * BR;
+        if (bt0 + BR > ta && bt0 < te) {
+          const int jj = bt0 >> a.block_shift;
+          const int phys = bt_s[jj - jb0];
+          if (phys >= 0) {
+            mine = true;
+            x = h * 64;
+            y = (phys * a.num_kv_heads + kvh) * a.block_size + (bt0 - (jj << a.block_shift));
+            dst = s * T::STAGE_BYTES + isv * T::KV_BYTES + h * T::HALF_BYTES + j * BR * 128;
+          }
+        }
+      }
+      const uint32_t nload = __popc(__ballot_sync(FULL, mine));
+      if (lane == 0) mbar_arrive_expect_tx(smem_u32(&bars[s]), nload * box_bytes);
+      __syncwarp();
+      if (mine)
+        tma_load_2d(smem_u32(smem) + dst, isv ? static_cast<const void*>(&tmv)
+                                              : static_cast<const void*>(&tmk),
+                    x, y, smem_u32(&bars[s]));
+      issued = k + 1;
+    }
+    if (lane == 0) {
+      for (int k = max(0, issued - NSTAGE); k < issued; ++k)
+        mbar_wait(smem_u32(&bars[k % NSTAGE]), (k / NSTAGE) & 1);
+    }
+    __syncwarp();
+  } else {
+    // ----------------------------- compute warps ---------------------------
+    const int cw = warp - 1;
+    const int mt = cw % NMT;
+    const int slice = cw / NMT;
+    const int nslice = (NCW - 1 - mt) / NMT + 1;
+    const int quad = lane >> 2, qi = lane & 3;
+    const int ra = mt * 16 + quad, rb = ra + 8;  // slab-local rows of this thread
+    int lo_a = INT_MAX, hi_a = INT_MIN, lo_b = INT_MAX, hi_b = INT_MIN;
+    if (ra < Rs) query_range(S, L, (row0 + ra) / a.group, w, lo_a, hi_a);
+    if (rb < Rs) query_range(S, L, (row0 + rb) / a.group, w, lo_b, hi_b);
+    int lo_max, hi_min, dummy;
+    query_range(S, L, L - 1, w, lo_max, dummy);  // the last token sees the latest start
+    query_range(S, L, 0, w, dummy, hi_min);      // the first token sees the earliest end
+
+    // Q as A fragments (bf16, exact); the scale is applied to the fp32 scores.
+    uint32_t qa[T::KSTEPS][4];
+    {
+      const uint32_t* qrow[2] = {nullptr, nullptr};
+      const int rows[2] = {ra, rb};
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        if (rows[e] < Rs) {
+          const int rr = row0 + rows[e];
+          const int i = rr / a.group, j = rr - (rr / a.group) * a.group;
+          qrow[e] = reinterpret_cast<const uint32_t*>(
+              a.q + ((size_t)(qoff + i) * a.num_q_heads + (size_t)kvh * a.group + j) * D);
+        }
+      }
+#pragma unroll
+      for (int ks = 0; ks < T::KSTEPS; ++ks) {
+        const int col2 = ks * 8 + qi;  // bf16-pair index of column ks*16 + 2*qi
+        qa[ks][0] = qrow[0] ? __ldg(qrow[0] + col2) : 0u;
+        qa[ks][1] = qrow[1] ? __ldg(qrow[1] + col2) : 0u;
+        qa[ks][2] = qrow[0] ? __ldg(qrow[0] + col2 + 4) : 0u;
+        qa[ks][3] = qrow[1] ? __ldg(qrow[1] + col2 + 4) : 0u;
+      }
+    }
+
+    float o[T::NT][4];
+#pragma unroll
+    for (int n = 0; n < T::NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    float m_a = kNegInf, m_b = kNegInf, l_a = 0.f, l_b = 0.f;
+
+    for (int k = 0; k < nst; ++k) {
+      const int s = k % NSTAGE;
+      const bool got = mbar_wait(smem_u32(&bars[s]), (k / NSTAGE) & 1);
+      if (!__all_sync(FULL, got)) break;
+      const uint32_t Ks = smem_u32(smem + s * T::STAGE_BYTES);
+      const uint32_t Vs = Ks + T::KV_BYTES;
+      const int c0 = p0 + k * TS;
+      const bool all_valid = (c0 >= lo_max) && (c0 + TS <= hi_min);
+      const bool boundary = (c0 < ulo) || (c0 + TS > p1);
+
+      for (int ch = slice; ch < TS / 16; ch += nslice) {
+        const int tb = ch * 16;
+        float sc[2][4];
+#pragma unroll
+        for (int n = 0; n < 2; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < T::KSTEPS; ++ks) {
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(Ks + swz(tb + ((lane >> 4) << 3) + (lane & 7), ks * 2 + ((lane >> 3) & 1)), b0,
+                  b1, b2, b3);
+          mma_bf16_16816(sc[0], qa[ks], b0, b1);
+          mma_bf16_16816(sc[1], qa[ks], b2, b3);
+        }
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sc[n][e] *= a.scale_log2;
+        if (!all_valid) {
+#pragma unroll
+          for (int n = 0; n < 2; ++n)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int t = c0 + tb + n * 8 + 2 * qi + (e & 1);
+              const bool ok = (e < 2) ? (t >= lo_a && t < hi_a) : (t >= lo_b && t < hi_b);
+              sc[n][e] = ok ? sc[n][e] : kNegInf;
+            }
+        }
+        float mx_a = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
+        float mx_b = fmaxf(fmaxf(sc[0][2], sc[0][3]), fmaxf(sc[1][2], sc[1][3]));
+        mx_a = fmaxf(mx_a, __shfl_xor_sync(FULL, mx_a, 1));
+        mx_a = fmaxf(mx_a, __shfl_xor_sync(FULL, mx_a, 2));
+        mx_b = fmaxf(mx_b, __shfl_xor_sync(FULL, mx_b, 1));
+        mx_b = fmaxf(mx_b, __shfl_xor_sync(FULL, mx_b, 2));
+        const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
+        const float mu_a = (mn_a == kNegInf) ? 0.f : mn_a;
+        const float mu_b = (mn_b == kNegInf) ? 0.f : mn_b;
+        const float al_a = (mn_a == kNegInf) ? 1.f : ex2(m_a - mu_a);
+        const float al_b = (mn_b == kNegInf) ? 1.f : ex2(m_b - mu_b);
+        m_a = mn_a;
+        m_b = mn_b;
+        float p[2][4];
+#pragma unroll
+        for (int n = 0; n < 2; ++n) {
+          p[n][0] = ex2(sc[n][0] - mu_a);
+          p[n][1] = ex2(sc[n][1] - mu_a);
+          p[n][2] = ex2(sc[n][2] - mu_b);
+          p[n][3] = ex2(sc[n][3] - mu_b);
+        }
+        l_a = l_a * al_a + (p[0][0] + p[0][1] + p[1][0] + p[1][1]);
+        l_b = l_b * al_b + (p[0][2] + p[0][3] + p[1][2] + p[1][3]);
+        if (__any_sync(FULL, al_a != 1.f || al_b != 1.f)) {
+#pragma unroll
+          for (int n = 0; n < T::NT; ++n) {
+            o[n][0] *= al_a;
+            o[n][1] *= al_a;
+            o[n][2] *= al_b;
+            o[n][3] *= al_b;
+          }
+        }
+        const uint32_t pa[4] = {pack_bf16x2(p[0][0], p[0][1]), pack_bf16x2(p[0][2], p[0][3]),
+                                pack_bf16x2(p[1][0], p[1][1]), pack_bf16x2(p[1][2], p[1][3])};
+        uint32_t mk_lo = 0xffffffffu, mk_hi = 0xffffffffu;
+        if (boundary) {
+          const int t = c0 + tb + 2 * qi;
+          auto in = [&](int u) { return u >= ulo && u < p1; };
+          mk_lo = (in(t) ? 0x0000ffffu : 0u) | (in(t + 1) ? 0xffff0000u : 0u);
+          mk_hi = (in(t + 8) ? 0x0000ffffu : 0u) | (in(t + 9) ? 0xffff0000u : 0u);
+        }
+#pragma unroll
+        for (int dp = 0; dp < T::NT / 2; ++dp) {
+          uint32_t v0, v1, v2, v3;
+          ldsm_x4_t(Vs + swz(tb + (((lane >> 3) & 1) << 3) + (lane & 7), dp * 2 + (lane >> 4)), v0,
+                    v1, v2, v3);
+          v0 &= mk_lo;
+          v1 &= mk_hi;
+          v2 &= mk_lo;
+          v3 &= mk_hi;
+          mma_bf16_16816(o[2 * dp], pa, v0, v1);
+          mma_bf16_16816(o[2 * dp + 1], pa, v2, v3);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars[NSTAGE + s]));
+    }
+
+    named_bar_sync(1, NCW * 32);
+#pragma unroll
+    for (int n = 0; n < T::NT; ++n) {
+      const int d = n * 8 + 2 * qi;
+      *reinterpret_cast<float2*>(comb_acc + (cw * 16 + quad) * D + d) = make_float2(o[n][0], o[n][1]);
+      *reinterpret_cast<float2*>(comb_acc + (cw * 16 + quad + 8) * D + d) =
+          make_float2(o[n][2], o[n][3]);
+    }
+    l_a += __shfl_xor_sync(FULL, l_a, 1);
+    l_a += __shfl_xor_sync(FULL, l_a, 2);
+    l_b += __shfl_xor_sync(FULL, l_b, 1);
+    l_b += __shfl_xor_sync(FULL, l_b, 2);
+    if (qi == 0) {
+      comb_l[cw * 16 + quad] = l_a;
+      comb_l[cw * 16 + quad + 8] = l_b;
+      comb_m[cw * 16 + quad] = m_a;
+      comb_m[cw * 16 + quad + 8] = m_b;
+    }
+  }
+  __syncthreads();
+
+  // ----------------- merge the compute warps' partials --------------------
+  for (int idx = threadIdx.x; idx < Rs * D; idx += blockDim.x) {
+    const int rloc = idx / D;
+    const int d = idx - rloc * D;
+    const int mti = rloc >> 4, r16 = rloc & 15;
+    float M = kNegInf;
+    for (int c = mti; c < NCW; c += NMT) M = fmaxf(M, comb_m[c * 16 + r16]);
+    float Z = 0.f, O = 0.f;
+    if (M != kNegInf) {
+      for (int c = mti; c < NCW; c += NMT) {
+        const float sc = ex2(comb_m[c * 16 + r16] - M);
+        Z += sc * comb_l[c * 16 + r16];
+        O += sc * comb_acc[(c * 16 + r16) * D + d];
+      }
+    }
+    const int rr = row0 + rloc;
+    if (nparts == 1) {
+      const int i = rr / a.group, j = rr - (rr / a.group) * a.group;
+      a.dst[((size_t)(qoff + i) * a.num_q_heads + (size_t)kvh * a.group + j) * D + d] =
+          __float2bfloat16_rn(O / Z);
+    } else {
+      const size_t base =
+          ((size_t)(b * a.num_kv_heads + kvh) * a.max_parts + part) * a.max_rows + rr;
+      a.ws_o[base * D + d] = Z > 0.f ? O / Z : 0.f;
+      if (d == 0) a.ws_lse[base] = Z > 0.f ? M + lg2(Z) : kNegInf;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Log-sum-exp reduce (ExecuTorch PR #18759, the split-K reduce kernel):
 // per (row, kv head, batch row): M = max_p lse_p, w_p = 2^(lse_p - M),
 // dst = sum_p w_p O_p / sum_p w_p.  Partials are normalised, so the weights
@@ -560,7 +913,55 @@ int occupancy_fma_t(size_t smem) {
   return n;
 }
 
+template <int D, int NCW, int NSTAGE>
+cudaError_t launch_mma_t(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
+                         dim3 grid, size_t smem, cudaStream_t stream) {
+  auto kern = pa_partition_mma_kernel<D, NCW, NSTAGE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, 32 * (NCW + 1), smem, stream>>>(a, tk, tv);
+  return cudaGetLastError();
+}
+
+template <int D, int NCW, int NSTAGE>
+int occupancy_mma_t(size_t smem) {
+  auto kern = pa_partition_mma_kernel<D, NCW, NSTAGE>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+      cudaSuccess)
+    return 0;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 32 * (NCW + 1), smem) != cudaSuccess)
+    return 0;
+  return n;
+}
+
 }  // namespace
+
+size_t mma_smem_bytes(int head_dim, int stages, int part_tokens, int block_size) {
+  const size_t ring = (size_t)stages * 2 * TS * head_dim * 2;
+  const size_t nbt = (size_t)part_tokens / block_size + 2;
+  return 1024 + ring + 2 * (size_t)stages * sizeof(uint64_t) + nbt * sizeof(int);
+}
+
+#define PA_MMA_DISPATCH(CALL)                                                       \
+  if (k.head_dim == 128 && k.consumer_warps == 4 && k.stages == 3) CALL(128, 4, 3); \
+  if (k.head_dim == 64 && k.consumer_warps == 4 && k.stages == 4) CALL(64, 4, 4);
+
+cudaError_t launch_partition_mma(const DecodeArgs& a, const KernelShape& k, const CUtensorMap& tk,
+                                 const CUtensorMap& tv, dim3 grid, size_t smem,
+                                 cudaStream_t stream) {
+#define PA_CALL(D, N, S) return launch_mma_t<D, N, S>(a, tk, tv, grid, smem, stream)
+  PA_MMA_DISPATCH(PA_CALL)
+#undef PA_CALL
+  return cudaErrorInvalidValue;
+}
+
+int occupancy_partition_mma(const KernelShape& k, size_t smem) {
+#define PA_CALL(D, N, S) return occupancy_mma_t<D, N, S>(smem)
+  PA_MMA_DISPATCH(PA_CALL)
+#undef PA_CALL
+  return 0;
+}
 
 size_t fma_smem_bytes(int head_dim, int stages, int part_tokens, int block_size) {
   const size_t ring = (size_t)stages * 2 * TS * head_dim * 2;

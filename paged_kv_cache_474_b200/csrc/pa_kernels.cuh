@@ -4,6 +4,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -51,6 +52,18 @@ cudaError_t launch_partition_fma(const DecodeArgs& a, const KernelShape& k, dim3
 
 // Occupancy (CTAs per SM) of an FMA partition-kernel instance.
 int occupancy_partition_fma(const KernelShape& k, size_t smem);
+
+// Dynamic shared memory of the tensor-core partition kernel.
+size_t mma_smem_bytes(int head_dim, int stages, int part_tokens, int block_size);
+
+// Launches the tensor-core partition kernel; tk / tv are 2-D tiled maps of
+// the K and V caches viewed as [rows][head_dim] with 64 x box-rows boxes and
+// the 128-byte swizzle.
+cudaError_t launch_partition_mma(const DecodeArgs& a, const KernelShape& k, const CUtensorMap& tk,
+                                 const CUtensorMap& tv, dim3 grid, size_t smem,
+                                 cudaStream_t stream);
+
+int occupancy_partition_mma(const KernelShape& k, size_t smem);
 
 // Launches the log-sum-exp reduce over (rows, kv heads, batch).
 cudaError_t launch_reduce(const DecodeArgs& a, cudaStream_t stream);

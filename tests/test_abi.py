@@ -156,12 +156,42 @@ def test_plan_forced_partitions_and_workspace_formula():
 
 
 def test_plan_row_slabs_for_many_rows():
-    info = plan(batch=4, num_q_heads=64, num_kv_heads=8, head_dim=128, num_blocks=400,
-                max_blocks_per_seq=64, bs=1024, max_span_hint=65536, max_query_len_hint=4)
-    assert info.max_rows == 32 and info.slab_rows == 32 and info.grid_y == 8
-    big = plan(batch=2, num_q_heads=64, num_kv_heads=4, head_dim=128, num_blocks=400,
-               max_blocks_per_seq=64, bs=1024, max_span_hint=65536, max_query_len_hint=5)
-    assert big.max_rows == 80 and big.grid_y == 4 * 3
+    kw = dict(batch=4, num_q_heads=64, num_kv_heads=8, head_dim=128, num_blocks=400,
+              max_blocks_per_seq=64, bs=1024, max_span_hint=65536, max_query_len_hint=4)
+    mma = plan(**kw)
+    assert mma.variant == pa.PA_VARIANT_MMA
+    assert mma.max_rows == 32 and mma.slab_rows == 64 and mma.grid_y == 8
+    fma = plan(force_variant=pa.PA_VARIANT_FMA, **kw)
+    assert fma.max_rows == 32 and fma.slab_rows == 32 and fma.grid_y == 8
+    kw.update(num_kv_heads=4, max_query_len_hint=5, batch=2)
+    big = plan(**kw)
+    assert big.max_rows == 80 and big.grid_y == 4 * 2
+    big_fma = plan(force_variant=pa.PA_VARIANT_FMA, **kw)
+    assert big_fma.grid_y == 4 * 3
+
+
+def test_plan_variant_follows_row_density():
+    # group x queryLen rows: 4 -> CUDA-core FMA, 8 and more -> tensor-core tiles
+    sparse = plan(batch=32, num_q_heads=32, num_kv_heads=8, head_dim=128, num_blocks=20000,
+                  max_blocks_per_seq=512, max_span_hint=8192)
+    dense = plan(batch=1, num_q_heads=8, num_kv_heads=1, head_dim=128, num_blocks=8193,
+                 max_blocks_per_seq=8192, max_span_hint=131072)
+    mtp = plan(batch=2, num_q_heads=8, num_kv_heads=4, head_dim=64, num_blocks=100,
+               max_blocks_per_seq=50, max_span_hint=700, max_query_len_hint=4)
+    assert sparse.variant == pa.PA_VARIANT_FMA
+    assert dense.variant == pa.PA_VARIANT_MMA and mtp.variant == pa.PA_VARIANT_MMA
+    forced = plan(batch=1, num_q_heads=8, num_kv_heads=1, head_dim=128, num_blocks=8193,
+                  max_blocks_per_seq=8192, max_span_hint=131072, force_variant=pa.PA_VARIANT_FMA)
+    assert forced.variant == pa.PA_VARIANT_FMA
+
+
+def test_plan_rejects_tensor_maps_beyond_32bit_rows():
+    rc, _ = pa.pa_plan(base_params(num_blocks=1 << 22, num_kv_heads=2, num_q_heads=16,
+                                   force_variant=pa.PA_VARIANT_MMA), 1024, 148, 2)
+    assert rc == pa.PA_ERR_UNSUPPORTED
+    rc, info = pa.pa_plan(base_params(num_blocks=1 << 22, num_kv_heads=2, num_q_heads=16,
+                                      max_query_len_hint=2), 1024, 148, 2)
+    assert rc == pa.PA_OK and info.variant == pa.PA_VARIANT_FMA
 
 
 def test_plan_caps_partition_at_the_table_cache():

@@ -66,45 +66,71 @@ def scaled(cfg, seed=1):
     raise ValueError(cfg)
 
 
+VARIANTS = [pa.PA_VARIANT_AUTO, pa.PA_VARIANT_FMA, pa.PA_VARIANT_MMA]
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
 @pytest.mark.parametrize("cfg", [2, 3, 4, 5])
 @pytest.mark.parametrize("parts", [0, 1, 5])
-def test_scaled_named_workloads(cfg, parts):
+def test_scaled_named_workloads(cfg, parts, variant):
     wl = scaled(cfg)
-    out = pa.decode(dev(wl), force_partitions=parts)
-    check_full(wl, out, f"scaled cfg{cfg} parts={parts}")
+    out = pa.decode(dev(wl), force_partitions=parts, force_variant=variant)
+    check_full(wl, out, f"scaled cfg{cfg} parts={parts} variant={variant}")
 
 
+def test_dispatcher_picks_fma_for_sparse_rows_and_mma_for_dense_tiles():
+    _, p2 = pa.pa_plan(pa.params_for(dev(scaled(2))), 16)
+    _, p4 = pa.pa_plan(pa.params_for(dev(scaled(4))), 16)
+    _, p5 = pa.pa_plan(pa.params_for(dev(scaled(5))), 1024)
+    assert p2.variant == pa.PA_VARIANT_FMA
+    assert p4.variant == pa.PA_VARIANT_MMA and p5.variant == pa.PA_VARIANT_MMA
+
+
+@pytest.mark.parametrize("variant", [pa.PA_VARIANT_FMA, pa.PA_VARIANT_MMA])
 @pytest.mark.parametrize("parts", [1, 2, 3, 7, 64, 200])
-def test_split_k_invariance(parts):
+def test_split_k_invariance(parts, variant):
     wl = make_workload(seq_lens=[5000, 3333, 77], query_lens=[1, 3, 2], num_q_heads=8,
                        num_kv_heads=2, head_dim=128, block_size=16, window=0, seed=7)
     d = dev(wl)
-    out = pa.decode(d, force_partitions=parts)
+    out = pa.decode(d, force_partitions=parts, force_variant=variant)
     check_full(wl, out, f"parts={parts}")
-    base = pa.decode(d, force_partitions=1).float()
+    base = pa.decode(d, force_partitions=1, force_variant=variant).float()
     assert torch.max(torch.abs(out.float() - base)).item() < 2e-2
 
 
+@pytest.mark.parametrize("variant", VARIANTS)
 @pytest.mark.parametrize("head_dim", [64, 128])
 @pytest.mark.parametrize("block_size", [16, 32, 64, 256, 1024])
-def test_head_dims_and_block_sizes(head_dim, block_size):
+def test_head_dims_and_block_sizes(head_dim, block_size, variant):
     wl = make_workload(seq_lens=[1, 17, 64, 65, 1500, 2049], query_lens=[1, 1, 2, 1, 4, 1],
                        num_q_heads=8, num_kv_heads=4, head_dim=head_dim,
                        block_size=block_size, window=0, seed=head_dim + block_size)
-    out = pa.decode(dev(wl))
-    check_full(wl, out, f"D={head_dim} BS={block_size}")
+    out = pa.decode(dev(wl), force_variant=variant)
+    check_full(wl, out, f"D={head_dim} BS={block_size} variant={variant}")
 
 
+@pytest.mark.parametrize("variant", [pa.PA_VARIANT_FMA, pa.PA_VARIANT_MMA])
+@pytest.mark.parametrize("group,qlen", [(1, 1), (2, 3), (8, 1), (8, 4), (16, 5), (64, 1)])
+def test_row_tiles_and_slabs(group, qlen, variant):
+    # rows per kv head from 1 to 80: padding rows, several M tiles, several slabs
+    wl = make_workload(seq_lens=[700, 64, 1999], query_lens=[qlen, min(qlen, 2), qlen],
+                       num_q_heads=2 * group, num_kv_heads=2, head_dim=128, block_size=16,
+                       window=0, seed=group * 10 + qlen)
+    out = pa.decode(dev(wl), force_variant=variant)
+    check_full(wl, out, f"group={group} qlen={qlen} variant={variant}")
+
+
+@pytest.mark.parametrize("variant", VARIANTS)
 @pytest.mark.parametrize("window", [1, 2, 5, 16, 100, 4096])
-def test_gllm_window_batch(window):
+def test_gllm_window_batch(window, variant):
     # gllm PR #116 "Verification": a 5-token prefill chunk over a 300-token
     # context plus a decode row over 40, windows 16, 100 and 4096 (and the
     # CPU test's small windows), here with GQA.
     wl = make_workload(seq_lens=[300, 40], query_lens=[5, 1], num_q_heads=8,
                        num_kv_heads=2, head_dim=64, block_size=16, window=window,
                        seed=window)
-    out = pa.decode(dev(wl))
-    check_full(wl, out, f"window={window}")
+    out = pa.decode(dev(wl), force_variant=variant)
+    check_full(wl, out, f"window={window} variant={variant}")
 
 
 def test_window_one_returns_own_value():
@@ -141,7 +167,8 @@ def test_rows_without_queries_and_empty_batch():
     assert rc == pa.PA_OK
 
 
-def test_garbage_outside_spans_is_never_read():
+@pytest.mark.parametrize("variant", [pa.PA_VARIANT_FMA, pa.PA_VARIANT_MMA])
+def test_garbage_outside_spans_is_never_read(variant):
     # Slots past each row's last token, the spare block and unused table
     # entries hold NaN / out-of-range values; outputs must not see them.
     wl = make_workload(seq_lens=[37, 50, 1], query_lens=[1, 3, 1], num_q_heads=4,
@@ -159,8 +186,25 @@ def test_garbage_outside_spans_is_never_read():
         if blk not in used:
             wl.k_cache[blk] = float("nan")
             wl.v_cache[blk] = float("nan")
-    out = pa.decode(dev(wl))
-    assert_close(out.float().cpu().numpy(), ref, "garbage outside spans")
+    out = pa.decode(dev(wl), force_variant=variant)
+    assert_close(out.float().cpu().numpy(), ref, f"garbage outside spans variant={variant}")
+
+
+@pytest.mark.parametrize("variant", [pa.PA_VARIANT_FMA, pa.PA_VARIANT_MMA])
+def test_windowed_garbage_before_the_window_is_never_read(variant):
+    # Positions before each row's window start hold NaN: a window that starts
+    # mid-block must still never let them into the output.
+    wl = make_workload(seq_lens=[1000, 333, 77], query_lens=[3, 1, 2], num_q_heads=8,
+                       num_kv_heads=2, head_dim=128, block_size=16, window=50, seed=19)
+    ref = oracle.decode(problem(wl))
+    for b, (S, L) in enumerate(zip(wl.seq_lens.tolist(), wl.query_lens.tolist())):
+        first = max(0, S - L + 1 - 50)
+        for t in range(first):
+            blk = int(wl.block_tables[b, t // 16])
+            wl.k_cache[blk, :, t % 16] = float("nan")
+            wl.v_cache[blk, :, t % 16] = float("nan")
+    out = pa.decode(dev(wl), force_variant=variant)
+    assert_close(out.float().cpu().numpy(), ref, f"window garbage variant={variant}")
 
 
 def test_no_hints_path_matches_hinted():
