@@ -195,6 +195,38 @@ size_t pa_host_workspace_size(const pa_params *params, int kvBlockSize, int wind
                               const int32_t *seqLens_host, const int32_t *queryLens_host);
 
 /*
+ * pa_decode_noalloc -- pa_decode for callers that cannot allocate device
+ * memory.  (The pages have no counterpart: this is a library convenience.)
+ *
+ * pa_decode needs a caller-allocated workspace for its split-K partials.
+ * Callers that cannot call cudaMalloc -- code running under another
+ * framework's allocator, plugins handed only input and output buffers, hot
+ * paths that must not allocate -- use this entry point instead: the partials
+ * live in a static device array compiled into the library,
+ * PA_NOALLOC_SCRATCH_BYTES (32 MiB) per GPU, which every GPU that loads the
+ * library holds until the process exits.  Arguments are those of pa_decode;
+ * params->workspace and workspace_bytes are ignored.  The caller still
+ * passes every input and output.
+ *
+ *  - The first call on a device looks up the array's device address with
+ *    that device current; make it before any stream capture.
+ *  - All calls on a device share the array: calls whose kernels overlap on
+ *    the GPU race.  Nothing in it needs to start at zero; each call reads
+ *    only partials it wrote itself.
+ *  - A call whose partials need more than PA_NOALLOC_SCRATCH_BYTES returns
+ *    PA_ERR_WORKSPACE before launching anything (pa_last_error() gives the
+ *    bytes needed); tight hints keep the need small.  PA_ERR_CUDA if the
+ *    array's address cannot be obtained.
+ *  - It calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+#define PA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+int pa_decode_noalloc(void *dst, const void *q, const void *kCache, const void *vCache,
+                      const int32_t *blockTables, const int32_t *seqLens,
+                      const int32_t *queryLens, float scale, int window, int kvBlockSize,
+                      const pa_params *params, void *stream);
+
+/*
  * pa_extents_host -- the two hints pa_params takes, from host copies of the
  * lengths: *max_span = longest union span over rows with queryLen > 0 (the
  * row's visible positions [max(0, S-L+1-window), S) for window > 0, else

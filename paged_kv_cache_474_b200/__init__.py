@@ -88,6 +88,7 @@ SIGNATURES = {
     "pa_plan": (_I, [_PP, _I, _I, _I, ctypes.POINTER(pa_plan_info)]),
     "pa_visible_ranges": (_I, [_P, _P, _P, _P, _I, _P, _I, _P]),
     "pa_decode_host": (_I, [_P, _P, _P, _P, _P, _P, _P, _F, _I, _I, _PP, _P]),
+    "pa_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _F, _I, _I, _PP, _P]),
     "pa_host_workspace_size": (ctypes.c_size_t, [_PP, _I, _I, _P, _P]),
     "pa_extents_host": (_I, [_P, _P, _P, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I)]),
     "pa_device_status": (_I, [ctypes.POINTER(ctypes.c_uint), _I, _P]),
@@ -132,6 +133,18 @@ def pa_decode(dst, q, kCache, vCache, blockTables, seqLens, queryLens, scale,
     return _lib.pa_decode(dst, q, kCache, vCache, blockTables, seqLens,
                           queryLens, float(scale), int(window), int(kvBlockSize),
                           ctypes.byref(params), stream)
+
+
+def pa_decode_noalloc(dst, q, kCache, vCache, blockTables, seqLens, queryLens, scale,
+                      window, kvBlockSize, params, stream) -> int:
+    """pa_decode with the library's static scratch array instead of a caller
+    workspace (for callers that cannot allocate device memory)."""
+    return _lib.pa_decode_noalloc(dst, q, kCache, vCache, blockTables, seqLens,
+                                  queryLens, float(scale), int(window), int(kvBlockSize),
+                                  ctypes.byref(params), stream)
+
+
+PA_NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
 def pa_workspace_size(params, kvBlockSize) -> int:

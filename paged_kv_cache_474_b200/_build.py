@@ -14,7 +14,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libpagedattn.so")
-SOURCES = ["pa_kernels.cu", "pa_api.cu"]
+SOURCES = ["pa_kernels.cu", "pa_api.cu", "pa_noalloc.cu"]
 HEADERS = ["pa_device.cuh", "pa_kernels.cuh", "pa_span.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
