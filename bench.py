@@ -71,10 +71,28 @@ class ClockSampler:
         self.proc = None
         self.lines = []
 
+    def _smi_id(self):
+        """nvidia-smi id of this process's CUDA device (matched by UUID, since
+        CUDA_VISIBLE_DEVICES may renumber devices)."""
+        try:
+            import torch
+            want = str(torch.cuda.get_device_properties(self.index).uuid).lower()
+            want = want.replace("gpu-", "").replace("-", "")
+            out = subprocess.run(["nvidia-smi", "--query-gpu=index,uuid",
+                                  "--format=csv,noheader"], capture_output=True,
+                                 text=True, timeout=30).stdout
+            for ln in out.splitlines():
+                idx, uuid = [x.strip() for x in ln.split(",")]
+                if uuid.lower().replace("gpu-", "").replace("-", "") == want:
+                    return idx
+        except Exception:
+            pass
+        return str(self.index)
+
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                ["nvidia-smi", f"--id={self._smi_id()}", f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self._t = threading.Thread(target=self._read, daemon=True)
@@ -97,6 +115,7 @@ class ClockSampler:
 
     def summary(self):
         sm, smax, reasons = [], None, set()
+        note = "sampled every 100 ms over >= 1 s of the same calls just before and during the timed steps"
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ln in self.lines:
             parts = [x.strip() for x in ln.split(",")]
@@ -111,9 +130,9 @@ class ClockSampler:
                 if v.lower() == "active":
                     reasons.add(n)
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": [], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": [], "samples": 0, "note": note}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm), "note": note}
 
 
 # ------------------------------------------------------------ the GPU arm
@@ -180,26 +199,40 @@ def run_ours(args, rank, world, local_rank):
 
     for _ in range(args.warmup):
         step()
-    # kernel events must exist before the timed region
+    torch.cuda.synchronize()
+    # Clock sampling covers a pre-roll of the same calls (at least ~1 s of
+    # load, so nvidia-smi sees the clocks under this work) and the timed steps.
+    with ClockSampler(local_rank) as clocks:
+        t_pre = time.perf_counter()
+        while time.perf_counter() - t_pre < 1.0:
+            for _ in range(20):
+                step()
+            torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+    elapsed_ms = t0.elapsed_time(t1)
+    # Partition-kernel duration: the same steps again, with the library
+    # recording events just before and after the partition kernel (kept out
+    # of the timed region above so the reduce's early launch is undisturbed).
     kev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
     for a, b in kev:     # torch creates the CUDA event on its first record
         a.record(stream)
         b.record(stream)
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local_rank) as clocks:
-        t0.record(stream)
-        for k in range(args.steps):
-            step(kev[k])
-        t1.record(stream)
-        torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    elapsed_ms = t0.elapsed_time(t1)
+    for k in range(args.steps):
+        step(kev[k])
+    torch.cuda.synchronize()
     kern_ms = [a.elapsed_time(b) for a, b in kev]
     t = torch.tensor([elapsed_ms], dtype=torch.float64, device=device)
     if world > 1:
@@ -248,6 +281,8 @@ def run_ours(args, rank, world, local_rank):
                      "kernel": ("pa_partition_mma_kernel" if plan.variant == pa.PA_VARIANT_MMA
                                 else "pa_partition_fma_kernel"),
                      "kernel_us": round(kern_avg_ms * 1e3, 2),
+                     "kernel_timing": "CUDA events the library records around the partition "
+                                      "kernel, averaged over the timed steps re-run",
                      "traffic": traffic},
         "e2e": e2e,
         "gpu_launches": launches,

@@ -144,7 +144,9 @@ int pa_decode(void *dst, const void *q, const void *kCache, const void *vCache,
  * pa_workspace_size -- bytes of workspace pa_decode needs for these params
  * (split-K partial maxima/sums and outputs for max(1, P) partitions, the
  * allocation rule aiter PR #2914's review asks for).  Uses the hints; with a
- * zero span hint it assumes the longest row fills max_blocks_per_seq blocks.
+ * zero span hint it assumes the longest row fills max_blocks_per_seq blocks,
+ * with a zero query-length hint it assumes one query token per row (size the
+ * workspace from real hints when rows carry several query tokens).
  * Returns 0 when the call is one-shot; (size_t)-1 on invalid params.
  * Host only; needs a CUDA device only when num_sms is not fixed (it queries
  * the current device's SM count and occupancy).

@@ -272,7 +272,11 @@ def decode(wl, *, out=None, workspace=None, hints=True, force_variant=PA_VARIANT
     p = params_for(wl, workspace=workspace, hints=hints, force_variant=force_variant,
                    force_partitions=force_partitions)
     if workspace is None:
-        workspace = alloc_workspace(p, wl.block_size, device=wl.q.device)
+        # size the workspace from the real extents even when the call itself
+        # runs without hints (pa_decode then reads the lengths itself)
+        sizing = p if hints else params_for(wl, force_variant=force_variant,
+                                            force_partitions=force_partitions)
+        workspace = alloc_workspace(sizing, wl.block_size, device=wl.q.device)
         if workspace is not None:
             p.workspace = workspace.data_ptr()
             p.workspace_bytes = workspace.numel()

@@ -16,6 +16,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -107,6 +108,27 @@ int check_params(const pa_params* p, int bs) {
   return PA_OK;
 }
 
+// Resident CTAs per SM of a kernel instance, queried once per device.
+int cached_occupancy(bool mma, const pa::KernelShape& k, size_t smem) {
+  static std::mutex mu;
+  static std::map<std::vector<long long>, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  const std::vector<long long> key = {dev, mma, k.head_dim, k.consumer_warps, k.stages, k.n8,
+                                      (long long)smem};
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+  }
+  const int n = mma ? pa::occupancy_partition_mma(k, smem) : pa::occupancy_partition_fma(k, smem);
+  if (n > 0) {
+    std::lock_guard<std::mutex> lock(mu);
+    cache[key] = n;
+  }
+  return n;
+}
+
 struct Plan {
   pa_plan_info info;
   pa::KernelShape shape;
@@ -124,18 +146,26 @@ int make_plan(const pa_params* p, int bs, int span, int qlen, int num_sms, int c
   if ((long long)G * qlen > 4096)
     return fail(PA_ERR_UNSUPPORTED, "rows per kv head %lld exceed 4096", (long long)G * qlen);
   const int rmax = G * qlen;
-  // Variant: tensor-core tiles once the rows of a (row, kv head) unit fill a
-  // real tile (8 or more), CUDA-core FMA below that.  The tensor-core path
-  // addresses cache rows through a TMA map with 32-bit row coordinates.
+  // Variant: the tensor-core kernel puts the KV tokens on the MMA's M axis
+  // and the unit's rows on N (8 per tile), so it serves every row count; on
+  // B200 it beats the CUDA-core FMA kernel even at 4 rows (GQA group 4 in an
+  // 8-wide tile: 122 vs 181 us on the GQA decode workload), because one
+  // m16n8k16 replaces ~40 FMA-path instructions per token.  The FMA kernel
+  // stays for pools whose row count exceeds the TMA map's 32-bit
+  // coordinates, and on request.
   const bool rows_fit_tma =
       (long long)p->num_blocks * p->num_kv_heads * bs <= (long long)INT32_MAX;
   int variant = p->force_variant;
-  if (variant == PA_VARIANT_AUTO) variant = (rmax > 4 && rows_fit_tma) ? PA_VARIANT_MMA : PA_VARIANT_FMA;
+  if (variant == PA_VARIANT_AUTO) variant = rows_fit_tma ? PA_VARIANT_MMA : PA_VARIANT_FMA;
   if (variant == PA_VARIANT_MMA && !rows_fit_tma)
     return fail(PA_ERR_UNSUPPORTED, "KV pool rows exceed the tensor map's 32-bit coordinates");
   const bool mma = variant == PA_VARIANT_MMA;
   const int ncw = mma ? 4 : (rmax <= 16 ? 4 : 8);
-  const int slab_rows = mma ? 16 * ncw : 4 * ncw;
+  // tensor-core warps cover 8 rows (one n-tile) when the unit has <= 8 rows,
+  // else 16; a CTA covers up to 4 such tiles.
+  const int n8 = (mma && rmax > 8) ? 2 : 1;
+  pl.shape.n8 = n8;
+  const int slab_rows = mma ? 8 * n8 * ncw : 4 * ncw;
   const int nslab = (int)cdiv(rmax, slab_rows);
   pl.shape.head_dim = p->head_dim;
   pl.shape.consumer_warps = ncw;
@@ -152,8 +182,7 @@ int make_plan(const pa_params* p, int bs, int span, int qlen, int num_sms, int c
     if (rc) return rc;
   }
   if (ctas_per_sm <= 0) {
-    ctas_per_sm = mma ? pa::occupancy_partition_mma(pl.shape, smem_for(cap))
-                      : pa::occupancy_partition_fma(pl.shape, smem_for(cap));
+    ctas_per_sm = cached_occupancy(mma, pl.shape, smem_for(cap));
     if (ctas_per_sm <= 0)
       return fail(PA_ERR_CUDA, "occupancy query failed: %s", cudaGetErrorString(cudaGetLastError()));
   }
@@ -170,8 +199,10 @@ int make_plan(const pa_params* p, int bs, int span, int qlen, int num_sms, int c
     ptok = std::max<long long>(ptok, kMinPartTokens);
   }
   ptok = std::min<long long>(std::max<long long>(ptok, TS), cap);
+  // The reduce keeps one weight per partition in smem: at most 16384.
+  ptok = std::max<long long>(ptok, cdiv(cdiv((long long)span + TS - 1, 16384), TS) * TS);
   const long long max_parts = cdiv((long long)span + TS - 1, ptok);
-  if (max_parts > (1LL << 30)) return fail(PA_ERR_UNSUPPORTED, "too many partitions");
+  if (max_parts > 16384) return fail(PA_ERR_UNSUPPORTED, "too many partitions");
 
   pa_plan_info& in = pl.info;
   in.variant = variant;
@@ -215,9 +246,12 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D map of a KV cache viewed as [num_blocks * H_kv * BS rows][head_dim]
-// bf16: boxes of 64 elements (128 bytes, the swizzle span) x box_rows rows,
-// 128-byte swizzle.  Encodings are cached per (base, rows, head_dim, box_rows).
+// 3-D map of a KV cache viewed as (64 elements, rows, head_dim/64 halves):
+// element stride 1, row stride head_dim*2 bytes, half stride 128 bytes.  A
+// box of (64, box_rows, halves) lands in smem as [half][row][128 B] with the
+// 128-byte swizzle (the half stride is smaller than the row stride on purpose:
+// the box's halves become separate 128-byte-wide tiles).  Encodings are cached
+// per (base, rows, head_dim, box_rows).
 int kv_tensor_map(CUtensorMap* out, const void* base, long long rows, int head_dim, int box_rows) {
   struct Entry {
     const void* base;
@@ -237,16 +271,16 @@ int kv_tensor_map(CUtensorMap* out, const void* base, long long rows, int head_d
   }
   auto fn = encode_fn();
   if (!fn) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
-  const cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
-  const cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
-  const cuuint32_t estr[2] = {1u, 1u};
+  const cuuint64_t dims[3] = {64u, (cuuint64_t)rows, (cuuint64_t)(head_dim / 64)};
+  const cuuint64_t strides[2] = {(cuuint64_t)head_dim * 2, 128u};
+  const cuuint32_t box[3] = {64u, (cuuint32_t)box_rows, (cuuint32_t)(head_dim / 64)};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
   Entry e;
   e.base = base;
   e.rows = rows;
   e.d = head_dim;
   e.br = box_rows;
-  const CUresult r = fn(&e.map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+  const CUresult r = fn(&e.map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);

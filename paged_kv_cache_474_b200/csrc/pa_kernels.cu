@@ -13,6 +13,9 @@
 // (cp.async.bulk + mbarrier transaction counts); compute warps read each
 // staged K/V row once for every query row of the GQA group.
 #include <climits>
+#include <map>
+#include <mutex>
+#include <utility>
 
 #include <cuda.h>
 
@@ -68,7 +71,7 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 // lane, then the 4 probabilities are broadcast back for the PV update.
 // ---------------------------------------------------------------------------
 template <int D, int NCW, int NSTAGE>
-__global__ void __launch_bounds__(32 * (NCW + 1), 1)
+__global__ void __launch_bounds__(32 * (NCW + 1), (NCW <= 4 ? 2 : 1))
     pa_partition_fma_kernel(const __grid_constant__ DecodeArgs a) {
   using T = FmaTraits<D>;
   using C = CombineLayout<D, NCW>;
@@ -138,6 +141,9 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
   }
   const int qoff = row_token_offset(a.query_lens, b, lane);
   __syncthreads();
+  // Let the reduce grid launch now; it waits for this grid's completion
+  // before reading any partial.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   float* comb_acc = reinterpret_cast<float*>(smem);
   float* comb_l = comb_acc + C::ACC_FLOATS;
@@ -389,20 +395,26 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
 }
 
 // ---------------------------------------------------------------------------
-// Partition kernel, tensor-core variant (rows = GQA group x query tokens form
-// a dense tile: group x queryLen >= 8).
+// Partition kernel, tensor-core variant.
 //
 // Staging: the copy warp loads whole KV boxes (one block for 16/32/64-token
-// blocks, a 64-token slice of larger blocks) with 2-D tiled TMA copies and
-// the 128-byte swizzle, so each stage holds K then V as [D/64][64 tokens]
-// [128 B] with 16-byte chunk c of token t stored at chunk c ^ (t & 7): every
-// ldmatrix below reads 8 distinct bank groups.  Compute: each compute warp
-// owns a 16-row M tile (rows past the real ones are padding) and a slice of
-// the stage's 16-token chunks; S = Q K^T and O += P V run as m16n8k16 bf16
-// MMAs with fp32 accumulation, P staying in registers between the two.
-// Tokens a box brings in from outside the row's visible union (the head of
-// the first block, the tail of the last) get score -inf and their V lanes
-// are zeroed in registers, so uninitialised cache slots never reach O.
+// blocks, a 64-token slice of larger blocks) with one 3-D tiled TMA copy per
+// box and K/V, with the 128-byte swizzle.  A box lands as [D/64 halves]
+// [BR rows][128 B] with 16-byte chunk c of row r stored at chunk c ^ (r & 7),
+// so every ldmatrix below reads 8 distinct bank groups; a stage holds the K
+// boxes, then the V boxes, of 64 tokens.
+//
+// Compute, with the KV tokens as the MMA's M dimension and the unit's query
+// rows as N (8 rows per n-tile, so an 8-row GQA group is one dense tile):
+//   S^T[16 tok x 8 rows] += K[16 tok x 16 d] . Q^T[16 d x 8 rows]
+//   O^T[16 d x 8 rows]   += V^T[16 d x 16 tok] . P^T[16 tok x 8 rows]
+// K and V^T come from smem by ldmatrix (V transposed on the fly), Q^T sits in
+// registers for the whole partition, and P^T moves from the S^T accumulator
+// layout to the B-operand layout with one movmatrix per 8x8 block.  Each
+// thread's O^T columns are exactly the rows whose softmax statistics it
+// holds, so the online-softmax rescale needs no data movement.  Tokens a box
+// brings in from outside the row's visible union get score -inf and their V
+// lanes are zeroed in registers, so uninitialised cache slots never reach O.
 // ---------------------------------------------------------------------------
 template <int D>
 struct MmaTraits {
@@ -410,30 +422,42 @@ struct MmaTraits {
   static constexpr int HALF_BYTES = TS * 128;
   static constexpr int KV_BYTES = HALVES * HALF_BYTES;
   static constexpr int STAGE_BYTES = 2 * KV_BYTES;
-  static constexpr int KSTEPS = D / 16;
-  static constexpr int NT = D / 8;  // 8-wide output column tiles
+  static constexpr int KSTEPS = D / 16;  // 16-wide reduction steps over d
+  static constexpr int MD = D / 16;      // 16-dim M tiles of O^T
 };
 
-template <int D, int NCW>
+template <int D, int NCW, int N8>
 struct MmaCombine {
-  static constexpr int ACC_FLOATS = NCW * 16 * D;
-  static constexpr int L_FLOATS = NCW * 16;
-  static constexpr int M_FLOATS = NCW * 16;
+  static constexpr int RT = 8 * N8;  // rows per warp tile
+  static constexpr int ACC_FLOATS = NCW * RT * D;
+  static constexpr int L_FLOATS = NCW * RT;
+  static constexpr int M_FLOATS = NCW * RT;
   static constexpr int BYTES = (ACC_FLOATS + L_FLOATS + M_FLOATS) * 4;
 };
 
-// Byte offset of 16-byte chunk `chunk` (0 .. D/8-1) of stage token row t.
-__device__ __forceinline__ uint32_t swz(int t, int chunk) {
-  return (uint32_t)((chunk >> 3) * (TS * 128) + t * 128 + (((chunk & 7) ^ (t & 7)) << 4));
+// Byte offset, within a box, of 16-byte chunk `chunk` (0 .. D/8-1) of row lt
+// (lt < 16, relative to a 16-row aligned chunk start): half (chunk / 8) of the
+// box, row lt, chunk position swizzled by the row's low three bits.
+__device__ __forceinline__ uint32_t box_off(int lt, int chunk, int BR) {
+  return (uint32_t)((chunk >> 3) * BR * 128 + lt * 128 + (((chunk & 7) ^ (lt & 7)) << 4));
 }
 
-template <int D, int NCW, int NSTAGE>
-__global__ void __launch_bounds__(32 * (NCW + 1), 1)
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// Register caps keep 4 (one n-tile) or 3 (two n-tiles) warps per SM
+// sub-partition, so two CTAs fit per SM.
+template <int D, int NCW, int NSTAGE, int N8>
+__global__ void __maxnreg__(N8 == 1 ? 128 : 168)
     pa_partition_mma_kernel(const __grid_constant__ DecodeArgs a,
                             const __grid_constant__ CUtensorMap tmk,
                             const __grid_constant__ CUtensorMap tmv) {
   using T = MmaTraits<D>;
-  using C = MmaCombine<D, NCW>;
+  using C = MmaCombine<D, NCW, N8>;
+  constexpr int RT = C::RT;
   static_assert(C::BYTES <= NSTAGE * T::STAGE_BYTES, "combine area must fit in the ring");
 
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -475,14 +499,6 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
   const int jb0 = p0 >> a.block_shift;
   const int nbt = ((p1 - 1) >> a.block_shift) - jb0 + 1;
 
-  for (int i = threadIdx.x; i < nbt; i += blockDim.x) {
-    int phys = a.block_tables[(size_t)b * a.max_blocks_per_seq + jb0 + i];
-    if (phys < 0 || phys >= a.num_blocks) {
-      atomicOr(&g_pa_status, PA_DEV_BAD_BLOCK);
-      phys = -1;
-    }
-    bt_s[i] = phys;
-  }
   if (threadIdx.x == 0) {
     prefetch_tensormap(&tmk);
     prefetch_tensormap(&tmv);
@@ -492,20 +508,36 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
     }
     fence_mbar_init();
   }
-  const int qoff = row_token_offset(a.query_lens, b, lane);
   __syncthreads();
+  // Let the reduce grid launch now; it waits for this grid's completion
+  // before reading any partial.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   float* comb_acc = reinterpret_cast<float*>(smem);
   float* comb_l = comb_acc + C::ACC_FLOATS;
   float* comb_m = comb_l + C::L_FLOATS;
-  const int NMT = (Rs + 15) >> 4;  // 16-row M tiles in this slab
+  const int NRT = (Rs + RT - 1) / RT;  // row tiles in this slab
+
+  // A box is BR token rows of one (block, kv head): [D/64 halves][BR rows][128 B].
+  const int BR = min(a.block_size, TS);
+  const uint32_t box_bytes = (uint32_t)BR * 128u * T::HALVES;
+  int qoff = 0;
 
   if (warp == 0) {
     // ------------------------------ copy warp ------------------------------
-    const int BR = min(a.block_size, TS);  // rows per box
+    // This warp alone reads the partition's block-table slice, so the first
+    // copies go out without waiting for the compute warps' prologue.
+    for (int i = lane; i < nbt; i += 32) {
+      int phys = a.block_tables[(size_t)b * a.max_blocks_per_seq + jb0 + i];
+      if (phys < 0 || phys >= a.num_blocks) {
+        atomicOr(&g_pa_status, PA_DEV_BAD_BLOCK);
+        phys = -1;
+      }
+      bt_s[i] = phys;
+    }
+    __syncwarp();
     const int nbox = TS / BR;
-    const int nitem = nbox * 2 * T::HALVES;  // (box, K/V, half) per lane
-    const uint32_t box_bytes = (uint32_t)BR * 128u;
+    const int nitem = nbox * 2;  // (box, K/V) per lane
     int issued = 0;
     for (int k = 0; k < nst; ++k) {
       const int s = k % NSTAGE;
@@ -518,21 +550,18 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
       const int ta = max(c0, ulo), te = min(c0 + TS, p1);
       bool mine = false;
       uint32_t dst = 0;
-      int x = 0, y = 0, isv = 0;
+      int y = 0, isv = 0;
       if (lane < nitem) {
-        const int j = lane / (2 * T::HALVES);
-        const int rem = lane - j * (2 * T::HALVES);
-        isv = rem / T::HALVES;
-        const int h = rem - isv * T::HALVES;
+        const int j = lane >> 1;
+        isv = lane & 1;
         const int bt0 = c0 + j * BR;
         if (bt0 + BR > ta && bt0 < te) {
           const int jj = bt0 >> a.block_shift;
           const int phys = bt_s[jj - jb0];
           if (phys >= 0) {
             mine = true;
-            x = h * 64;
             y = (phys * a.num_kv_heads + kvh) * a.block_size + (bt0 - (jj << a.block_shift));
-            dst = s * T::STAGE_BYTES + isv * T::KV_BYTES + h * T::HALF_BYTES + j * BR * 128;
+            dst = s * T::STAGE_BYTES + isv * T::KV_BYTES + j * box_bytes;
           }
         }
       }
@@ -540,9 +569,9 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
       if (lane == 0) mbar_arrive_expect_tx(smem_u32(&bars[s]), nload * box_bytes);
       __syncwarp();
       if (mine)
-        tma_load_2d(smem_u32(smem) + dst, isv ? static_cast<const void*>(&tmv)
+        tma_load_3d(smem_u32(smem) + dst, isv ? static_cast<const void*>(&tmv)
                                               : static_cast<const void*>(&tmk),
-                    x, y, smem_u32(&bars[s]));
+                    0, y, 0, smem_u32(&bars[s]));
       issued = k + 1;
     }
     if (lane == 0) {
@@ -550,49 +579,62 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
         mbar_wait(smem_u32(&bars[k % NSTAGE]), (k / NSTAGE) & 1);
     }
     __syncwarp();
+    qoff = row_token_offset(a.query_lens, b, lane);
   } else {
     // ----------------------------- compute warps ---------------------------
     const int cw = warp - 1;
-    const int mt = cw % NMT;
-    const int slice = cw / NMT;
-    const int nslice = (NCW - 1 - mt) / NMT + 1;
+    const int rt = cw % NRT;
+    const int slice = cw / NRT;
+    const int nslice = (NCW - 1 - rt) / NRT + 1;
     const int quad = lane >> 2, qi = lane & 3;
-    const int ra = mt * 16 + quad, rb = ra + 8;  // slab-local rows of this thread
-    int lo_a = INT_MAX, hi_a = INT_MIN, lo_b = INT_MAX, hi_b = INT_MIN;
-    if (ra < Rs) query_range(S, L, (row0 + ra) / a.group, w, lo_a, hi_a);
-    if (rb < Rs) query_range(S, L, (row0 + rb) / a.group, w, lo_b, hi_b);
+    qoff = row_token_offset(a.query_lens, b, lane);
+    const int brs = a.block_shift < 6 ? a.block_shift : 6;  // log2(BR)
+    // lane parts of the ldmatrix row addresses (token row within the chunk,
+    // 16-byte chunk parity) for K (A operand) and V (A operand, transposed)
+    const int lt_k = (((lane >> 3) & 1) << 3) + (lane & 7), ck_k = lane >> 4;
+    const int lt_v = ((lane >> 4) << 3) + (lane & 7), ck_v = (lane >> 3) & 1;
     int lo_max, hi_min, dummy;
     query_range(S, L, L - 1, w, lo_max, dummy);  // the last token sees the latest start
     query_range(S, L, 0, w, dummy, hi_min);      // the first token sees the earliest end
 
-    // Q as A fragments (bf16, exact); the scale is applied to the fp32 scores.
-    uint32_t qa[T::KSTEPS][4];
-    {
-      const uint32_t* qrow[2] = {nullptr, nullptr};
-      const int rows[2] = {ra, rb};
+    // Q^T as B fragments (exact bf16): n-tile n holds warp-tile rows n*8..n*8+7;
+    // this thread feeds row n*8 + quad, dims ks*16 + 2*qi (+1) and +8 (+9).
+    uint32_t qb[T::KSTEPS][N8][2];
+    // Softmax statistics of the rows n*8 + 2*qi + j (j = 0, 1): the O^T columns
+    // this thread accumulates.
+    int lo_r[N8][2], hi_r[N8][2];
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        if (rows[e] < Rs) {
-          const int rr = row0 + rows[e];
-          const int i = rr / a.group, j = rr - (rr / a.group) * a.group;
-          qrow[e] = reinterpret_cast<const uint32_t*>(
-              a.q + ((size_t)(qoff + i) * a.num_q_heads + (size_t)kvh * a.group + j) * D);
-        }
+    for (int n = 0; n < N8; ++n) {
+      const int rq = rt * RT + n * 8 + quad;
+      const uint32_t* qp = nullptr;
+      if (rq < Rs) {
+        const int rr = row0 + rq;
+        const int i = rr / a.group, j = rr - (rr / a.group) * a.group;
+        qp = reinterpret_cast<const uint32_t*>(
+            a.q + ((size_t)(qoff + i) * a.num_q_heads + (size_t)kvh * a.group + j) * D);
       }
 #pragma unroll
       for (int ks = 0; ks < T::KSTEPS; ++ks) {
-        const int col2 = ks * 8 + qi;  // bf16-pair index of column ks*16 + 2*qi
-        qa[ks][0] = qrow[0] ? __ldg(qrow[0] + col2) : 0u;
-        qa[ks][1] = qrow[1] ? __ldg(qrow[1] + col2) : 0u;
-        qa[ks][2] = qrow[0] ? __ldg(qrow[0] + col2 + 4) : 0u;
-        qa[ks][3] = qrow[1] ? __ldg(qrow[1] + col2 + 4) : 0u;
+        qb[ks][n][0] = qp ? __ldg(qp + ks * 8 + qi) : 0u;
+        qb[ks][n][1] = qp ? __ldg(qp + ks * 8 + qi + 4) : 0u;
+      }
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int rs = rt * RT + n * 8 + 2 * qi + j;
+        lo_r[n][j] = INT_MAX;
+        hi_r[n][j] = INT_MIN;
+        if (rs < Rs) query_range(S, L, (row0 + rs) / a.group, w, lo_r[n][j], hi_r[n][j]);
       }
     }
 
-    float o[T::NT][4];
+    float o[T::MD][N8][4];
 #pragma unroll
-    for (int n = 0; n < T::NT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-    float m_a = kNegInf, m_b = kNegInf, l_a = 0.f, l_b = 0.f;
+    for (int md = 0; md < T::MD; ++md)
+#pragma unroll
+      for (int n = 0; n < N8; ++n) o[md][n][0] = o[md][n][1] = o[md][n][2] = o[md][n][3] = 0.f;
+    float m_r[N8][2], l_r[N8][2];
+#pragma unroll
+    for (int n = 0; n < N8; ++n) m_r[n][0] = m_r[n][1] = kNegInf, l_r[n][0] = l_r[n][1] = 0.f;
 
     for (int k = 0; k < nst; ++k) {
       const int s = k % NSTAGE;
@@ -606,65 +648,74 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
 
       for (int ch = slice; ch < TS / 16; ch += nslice) {
         const int tb = ch * 16;
-        float sc[2][4];
+        // the chunk's 16 tokens lie in one box (BR >= 16)
+        const uint32_t cbase = (uint32_t)((tb >> brs) * box_bytes + (tb & (BR - 1)) * 128);
+        // S^T = K Q^T; with one n-tile, two accumulator sets (even / odd d
+        // steps) halve the dependent MMA chain.
+        constexpr int NACC = N8 == 1 ? 2 : 1;
+        float sc[2][N8][4];
 #pragma unroll
-        for (int n = 0; n < 2; ++n) sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
+        for (int u = 0; u < 2; ++u)
+#pragma unroll
+          for (int n = 0; n < N8; ++n) sc[u][n][0] = sc[u][n][1] = sc[u][n][2] = sc[u][n][3] = 0.f;
 #pragma unroll
         for (int ks = 0; ks < T::KSTEPS; ++ks) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(Ks + swz(tb + ((lane >> 4) << 3) + (lane & 7), ks * 2 + ((lane >> 3) & 1)), b0,
-                  b1, b2, b3);
-          mma_bf16_16816(sc[0], qa[ks], b0, b1);
-          mma_bf16_16816(sc[1], qa[ks], b2, b3);
+          uint32_t ka[4];
+          ldsm_x4(Ks + cbase + box_off(lt_k, ks * 2 + ck_k, BR), ka[0], ka[1], ka[2], ka[3]);
+#pragma unroll
+          for (int n = 0; n < N8; ++n)
+            mma_bf16_16816(sc[ks % NACC][n], ka, qb[ks][n][0], qb[ks][n][1]);
         }
+        // element e of n-tile n: token tb + quad + 8*(e>>1), row n*8 + 2*qi + (e&1)
+        float p[N8][4];
+        bool any_rescale = false;
+        float al[N8][2];
 #pragma unroll
-        for (int n = 0; n < 2; ++n)
+        for (int n = 0; n < N8; ++n) {
+          float v[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) sc[n][e] *= a.scale_log2;
-        if (!all_valid) {
-#pragma unroll
-          for (int n = 0; n < 2; ++n)
+          for (int e = 0; e < 4; ++e) v[e] = (sc[0][n][e] + sc[1][n][e]) * a.scale_log2;
+          if (!all_valid) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int t = c0 + tb + n * 8 + 2 * qi + (e & 1);
-              const bool ok = (e < 2) ? (t >= lo_a && t < hi_a) : (t >= lo_b && t < hi_b);
-              sc[n][e] = ok ? sc[n][e] : kNegInf;
+              const int t = c0 + tb + quad + ((e >> 1) << 3);
+              v[e] = (t >= lo_r[n][e & 1] && t < hi_r[n][e & 1]) ? v[e] : kNegInf;
             }
-        }
-        float mx_a = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
-        float mx_b = fmaxf(fmaxf(sc[0][2], sc[0][3]), fmaxf(sc[1][2], sc[1][3]));
-        mx_a = fmaxf(mx_a, __shfl_xor_sync(FULL, mx_a, 1));
-        mx_a = fmaxf(mx_a, __shfl_xor_sync(FULL, mx_a, 2));
-        mx_b = fmaxf(mx_b, __shfl_xor_sync(FULL, mx_b, 1));
-        mx_b = fmaxf(mx_b, __shfl_xor_sync(FULL, mx_b, 2));
-        const float mn_a = fmaxf(m_a, mx_a), mn_b = fmaxf(m_b, mx_b);
-        const float mu_a = (mn_a == kNegInf) ? 0.f : mn_a;
-        const float mu_b = (mn_b == kNegInf) ? 0.f : mn_b;
-        const float al_a = (mn_a == kNegInf) ? 1.f : ex2(m_a - mu_a);
-        const float al_b = (mn_b == kNegInf) ? 1.f : ex2(m_b - mu_b);
-        m_a = mn_a;
-        m_b = mn_b;
-        float p[2][4];
+          }
 #pragma unroll
-        for (int n = 0; n < 2; ++n) {
-          p[n][0] = ex2(sc[n][0] - mu_a);
-          p[n][1] = ex2(sc[n][1] - mu_a);
-          p[n][2] = ex2(sc[n][2] - mu_b);
-          p[n][3] = ex2(sc[n][3] - mu_b);
-        }
-        l_a = l_a * al_a + (p[0][0] + p[0][1] + p[1][0] + p[1][1]);
-        l_b = l_b * al_b + (p[0][2] + p[0][3] + p[1][2] + p[1][3]);
-        if (__any_sync(FULL, al_a != 1.f || al_b != 1.f)) {
-#pragma unroll
-          for (int n = 0; n < T::NT; ++n) {
-            o[n][0] *= al_a;
-            o[n][1] *= al_a;
-            o[n][2] *= al_b;
-            o[n][3] *= al_b;
+          for (int j = 0; j < 2; ++j) {
+            float mx = fmaxf(v[j], v[j + 2]);
+            mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 4));
+            mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 8));
+            mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 16));
+            const float mn = fmaxf(m_r[n][j], mx);
+            const float mu = (mn == kNegInf) ? 0.f : mn;
+            al[n][j] = (mn == kNegInf) ? 1.f : ex2(m_r[n][j] - mu);
+            any_rescale |= (al[n][j] != 1.f);
+            m_r[n][j] = mn;
+            p[n][j] = ex2(v[j] - mu);
+            p[n][j + 2] = ex2(v[j + 2] - mu);
+            l_r[n][j] = l_r[n][j] * al[n][j] + (p[n][j] + p[n][j + 2]);
           }
         }
-        const uint32_t pa[4] = {pack_bf16x2(p[0][0], p[0][1]), pack_bf16x2(p[0][2], p[0][3]),
-                                pack_bf16x2(p[1][0], p[1][1]), pack_bf16x2(p[1][2], p[1][3])};
+        if (__any_sync(FULL, any_rescale)) {
+#pragma unroll
+          for (int md = 0; md < T::MD; ++md)
+#pragma unroll
+            for (int n = 0; n < N8; ++n) {
+              o[md][n][0] *= al[n][0];
+              o[md][n][1] *= al[n][1];
+              o[md][n][2] *= al[n][0];
+              o[md][n][3] *= al[n][1];
+            }
+        }
+        // P^T B fragments: the accumulator's 8x8 blocks transposed in registers.
+        uint32_t pb[N8][2];
+#pragma unroll
+        for (int n = 0; n < N8; ++n) {
+          pb[n][0] = movmatrix_trans(pack_bf16x2(p[n][0], p[n][1]));
+          pb[n][1] = movmatrix_trans(pack_bf16x2(p[n][2], p[n][3]));
+        }
         uint32_t mk_lo = 0xffffffffu, mk_hi = 0xffffffffu;
         if (boundary) {
           const int t = c0 + tb + 2 * qi;
@@ -673,16 +724,15 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
           mk_hi = (in(t + 8) ? 0x0000ffffu : 0u) | (in(t + 9) ? 0xffff0000u : 0u);
         }
 #pragma unroll
-        for (int dp = 0; dp < T::NT / 2; ++dp) {
-          uint32_t v0, v1, v2, v3;
-          ldsm_x4_t(Vs + swz(tb + (((lane >> 3) & 1) << 3) + (lane & 7), dp * 2 + (lane >> 4)), v0,
-                    v1, v2, v3);
-          v0 &= mk_lo;
-          v1 &= mk_hi;
-          v2 &= mk_lo;
-          v3 &= mk_hi;
-          mma_bf16_16816(o[2 * dp], pa, v0, v1);
-          mma_bf16_16816(o[2 * dp + 1], pa, v2, v3);
+        for (int md = 0; md < T::MD; ++md) {
+          uint32_t va[4];
+          ldsm_x4_t(Vs + cbase + box_off(lt_v, md * 2 + ck_v, BR), va[0], va[1], va[2], va[3]);
+          va[0] &= mk_lo;
+          va[1] &= mk_lo;
+          va[2] &= mk_hi;
+          va[3] &= mk_hi;
+#pragma unroll
+          for (int n = 0; n < N8; ++n) mma_bf16_16816(o[md][n], va, pb[n][0], pb[n][1]);
         }
       }
       __syncwarp();
@@ -690,23 +740,28 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
     }
 
     named_bar_sync(1, NCW * 32);
+    // O^T element (md, n, e): dim md*16 + quad + 8*(e>>1), row n*8 + 2*qi + (e&1)
 #pragma unroll
-    for (int n = 0; n < T::NT; ++n) {
-      const int d = n * 8 + 2 * qi;
-      *reinterpret_cast<float2*>(comb_acc + (cw * 16 + quad) * D + d) = make_float2(o[n][0], o[n][1]);
-      *reinterpret_cast<float2*>(comb_acc + (cw * 16 + quad + 8) * D + d) =
-          make_float2(o[n][2], o[n][3]);
-    }
-    l_a += __shfl_xor_sync(FULL, l_a, 1);
-    l_a += __shfl_xor_sync(FULL, l_a, 2);
-    l_b += __shfl_xor_sync(FULL, l_b, 1);
-    l_b += __shfl_xor_sync(FULL, l_b, 2);
-    if (qi == 0) {
-      comb_l[cw * 16 + quad] = l_a;
-      comb_l[cw * 16 + quad + 8] = l_b;
-      comb_m[cw * 16 + quad] = m_a;
-      comb_m[cw * 16 + quad + 8] = m_b;
-    }
+    for (int md = 0; md < T::MD; ++md)
+#pragma unroll
+      for (int n = 0; n < N8; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          comb_acc[(cw * RT + n * 8 + 2 * qi + (e & 1)) * D + md * 16 + quad + ((e >> 1) << 3)] =
+              o[md][n][e];
+#pragma unroll
+    for (int n = 0; n < N8; ++n)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        float l = l_r[n][j];
+        l += __shfl_xor_sync(FULL, l, 4);
+        l += __shfl_xor_sync(FULL, l, 8);
+        l += __shfl_xor_sync(FULL, l, 16);
+        if (quad == 0) {
+          comb_l[cw * RT + n * 8 + 2 * qi + j] = l;
+          comb_m[cw * RT + n * 8 + 2 * qi + j] = m_r[n][j];
+        }
+      }
   }
   __syncthreads();
 
@@ -714,15 +769,15 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
   for (int idx = threadIdx.x; idx < Rs * D; idx += blockDim.x) {
     const int rloc = idx / D;
     const int d = idx - rloc * D;
-    const int mti = rloc >> 4, r16 = rloc & 15;
+    const int rti = rloc / RT, rr8 = rloc - rti * RT;
     float M = kNegInf;
-    for (int c = mti; c < NCW; c += NMT) M = fmaxf(M, comb_m[c * 16 + r16]);
+    for (int c = rti; c < NCW; c += NRT) M = fmaxf(M, comb_m[c * RT + rr8]);
     float Z = 0.f, O = 0.f;
     if (M != kNegInf) {
-      for (int c = mti; c < NCW; c += NMT) {
-        const float sc = ex2(comb_m[c * 16 + r16] - M);
-        Z += sc * comb_l[c * 16 + r16];
-        O += sc * comb_acc[(c * 16 + r16) * D + d];
+      for (int c = rti; c < NCW; c += NRT) {
+        const float sc = ex2(comb_m[c * RT + rr8] - M);
+        Z += sc * comb_l[c * RT + rr8];
+        O += sc * comb_acc[(c * RT + rr8) * D + d];
       }
     }
     const int rr = row0 + rloc;
@@ -744,17 +799,25 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1)
 // per (row, kv head, batch row): M = max_p lse_p, w_p = 2^(lse_p - M),
 // dst = sum_p w_p O_p / sum_p w_p.  Partials are normalised, so the weights
 // carry each partition's softmax mass.
+//
+// One CTA per (row, kv head, batch row).  The CTA first loads every lse_p
+// (one coalesced pass), forms the weights in smem, then its warps sum w_p O_p
+// over interleaved partitions with four independent partial loads in flight
+// per lane, each lane owning D/32 consecutive dims; warps merge through smem.
+// Launched with programmatic stream serialization: it may be scheduled while
+// the partition kernel drains and waits on griddepcontrol before reading.
 // ---------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(256) pa_reduce_kernel(const __grid_constant__ DecodeArgs a) {
-  constexpr int NT = 256;
-  constexpr int DQ = D / 4;
-  constexpr int NPG = NT / DQ;
-  __shared__ float red[NT / 32];
-  __shared__ float4 pacc[NT];
-  __shared__ float s_bcast;
+__global__ void __launch_bounds__(512) pa_reduce_kernel(const __grid_constant__ DecodeArgs a) {
+  constexpr int VPL = D / 32;  // dims per lane
+  constexpr int BATCH = 4;     // partial loads in flight per lane
+  extern __shared__ float s_w[];  // [max_parts] weights
+  __shared__ float s_red[16];
+  __shared__ __align__(16) float s_acc[16][D];
+  __shared__ float s_M, s_Z;
   __shared__ int s_qoff;
 
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int rr = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int S = a.seq_lens[b];
   const int L = a.query_lens[b];
@@ -767,6 +830,7 @@ __global__ void __launch_bounds__(256) pa_reduce_kernel(const __grid_constant__ 
   if (nparts <= 1 || nparts > a.max_parts) return;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nw = blockDim.x >> 5;
   if (warp == 0) {
     const int q0 = row_token_offset(a.query_lens, b, lane);
     if (lane == 0) s_qoff = q0;
@@ -775,59 +839,87 @@ __global__ void __launch_bounds__(256) pa_reduce_kernel(const __grid_constant__ 
   const float* lse = a.ws_lse + ubase * a.max_rows + rr;
 
   float m = kNegInf;
-  for (int p = tid; p < nparts; p += NT) m = fmaxf(m, lse[(size_t)p * a.max_rows]);
+  for (int p = tid; p < nparts; p += blockDim.x) {
+    const float v = lse[(size_t)p * a.max_rows];
+    s_w[p] = v;
+    m = fmaxf(m, v);
+  }
 #pragma unroll
   for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
-  if (lane == 0) red[warp] = m;
+  if (lane == 0) s_red[warp] = m;
   __syncthreads();
   if (tid == 0) {
-    float x = red[0];
-    for (int i = 1; i < NT / 32; ++i) x = fmaxf(x, red[i]);
-    s_bcast = x;
+    float x = s_red[0];
+    for (int i = 1; i < nw; ++i) x = fmaxf(x, s_red[i]);
+    s_M = x;
   }
   __syncthreads();
-  const float M = s_bcast;
-  __syncthreads();
-
+  const float M = s_M;
   float z = 0.f;
-  for (int p = tid; p < nparts; p += NT) z += ex2(lse[(size_t)p * a.max_rows] - M);
+  for (int p = tid; p < nparts; p += blockDim.x) {
+    const float wt = ex2(s_w[p] - M);  // an empty partition (-inf) weighs 0
+    s_w[p] = wt;
+    z += wt;
+  }
 #pragma unroll
   for (int o = 16; o; o >>= 1) z += __shfl_xor_sync(FULL, z, o);
-  if (lane == 0) red[warp] = z;
-
-  const int dq = tid % DQ, pg = tid / DQ;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int p = pg; p < nparts; p += NPG) {
-    const float wt = ex2(lse[(size_t)p * a.max_rows] - M);
-    const float4 o =
-        *reinterpret_cast<const float4*>(a.ws_o + ((ubase + p) * a.max_rows + rr) * D + dq * 4);
-    acc.x += wt * o.x;
-    acc.y += wt * o.y;
-    acc.z += wt * o.z;
-    acc.w += wt * o.w;
-  }
-  pacc[tid] = acc;
   __syncthreads();
-  if (pg == 0) {
-    float Z = 0.f;
-    for (int i = 0; i < NT / 32; ++i) Z += red[i];
-    for (int g = 1; g < NPG; ++g) {
-      const float4 o = pacc[g * DQ + dq];
-      acc.x += o.x;
-      acc.y += o.y;
-      acc.z += o.z;
-      acc.w += o.w;
+  if (lane == 0) s_red[warp] = z;
+  __syncthreads();
+  if (tid == 0) {
+    float x = 0.f;
+    for (int i = 0; i < nw; ++i) x += s_red[i];
+    s_Z = x;
+  }
+
+  float acc[VPL];
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) acc[v] = 0.f;
+  const float* obase = a.ws_o + (ubase * a.max_rows + rr) * D + lane * VPL;
+  const size_t pstride = (size_t)a.max_rows * D;
+  for (int p0 = warp; p0 < nparts; p0 += BATCH * nw) {
+    float o[BATCH][VPL];
+#pragma unroll
+    for (int u = 0; u < BATCH; ++u) {
+      const int p = p0 + u * nw;
+      if (p < nparts) {
+        if constexpr (VPL == 4) {
+          const float4 t = *reinterpret_cast<const float4*>(obase + p * pstride);
+          o[u][0] = t.x, o[u][1] = t.y, o[u][2] = t.z, o[u][3] = t.w;
+        } else {
+          const float2 t = *reinterpret_cast<const float2*>(obase + p * pstride);
+          o[u][0] = t.x, o[u][1] = t.y;
+        }
+      } else {
+#pragma unroll
+        for (int v = 0; v < VPL; ++v) o[u][v] = 0.f;
+      }
     }
-    const float inv = 1.f / Z;
+#pragma unroll
+    for (int u = 0; u < BATCH; ++u) {
+      const int p = p0 + u * nw;
+      const float wt = p < nparts ? s_w[p] : 0.f;
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) acc[v] += wt * o[u][v];
+    }
+  }
+#pragma unroll
+  for (int v = 0; v < VPL; ++v) s_acc[warp][lane * VPL + v] = acc[v];
+  __syncthreads();
+  if (warp == 0) {
+    float out[VPL];
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) out[v] = 0.f;
+    for (int i = 0; i < nw; ++i)
+#pragma unroll
+      for (int v = 0; v < VPL; ++v) out[v] += s_acc[i][lane * VPL + v];
+    const float inv = 1.f / s_Z;
     const int i = rr / a.group, j = rr - (rr / a.group) * a.group;
-    __nv_bfloat16* dp =
-        a.dst + ((size_t)(s_qoff + i) * a.num_q_heads + (size_t)kvh * a.group + j) * D + dq * 4;
-    const __nv_bfloat162 lo2 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-    const __nv_bfloat162 hi2 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-    uint2 packed;
-    packed.x = *reinterpret_cast<const uint32_t*>(&lo2);
-    packed.y = *reinterpret_cast<const uint32_t*>(&hi2);
-    *reinterpret_cast<uint2*>(dp) = packed;
+    __nv_bfloat16* dp = a.dst + ((size_t)(s_qoff + i) * a.num_q_heads + (size_t)kvh * a.group + j) * D +
+                        lane * VPL;
+#pragma unroll
+    for (int v = 0; v < VPL; v += 2)
+      *reinterpret_cast<__nv_bfloat162*>(dp + v) = __floats2bfloat162_rn(out[v] * inv, out[v + 1] * inv);
   }
 }
 
@@ -892,10 +984,30 @@ __global__ void __launch_bounds__(1024) pa_ranges_kernel(int32_t* lo, int32_t* h
   }
 }
 
+// Sets a kernel's dynamic-smem limit and asks for the largest shared-memory
+// carveout (so two CTAs fit per SM), once per (device, kernel, size).
+cudaError_t ensure_smem_attrs(const void* kern, size_t smem) {
+  static std::mutex mu;
+  static std::map<std::pair<int, const void*>, size_t> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = done.find({dev, kern});
+  if (it != done.end() && it->second >= smem) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           (int)cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return e;
+  done[{dev, kern}] = smem;
+  return cudaSuccess;
+}
+
 template <int D, int NCW, int NSTAGE>
 cudaError_t launch_fma_t(const DecodeArgs& a, dim3 grid, size_t smem, cudaStream_t stream) {
   auto kern = pa_partition_fma_kernel<D, NCW, NSTAGE>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = ensure_smem_attrs(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   kern<<<grid, 32 * (NCW + 1), smem, stream>>>(a);
   return cudaGetLastError();
@@ -904,31 +1016,27 @@ cudaError_t launch_fma_t(const DecodeArgs& a, dim3 grid, size_t smem, cudaStream
 template <int D, int NCW, int NSTAGE>
 int occupancy_fma_t(size_t smem) {
   auto kern = pa_partition_fma_kernel<D, NCW, NSTAGE>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-      cudaSuccess)
-    return 0;
+  if (ensure_smem_attrs(reinterpret_cast<const void*>(kern), smem) != cudaSuccess) return 0;
   int n = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 32 * (NCW + 1), smem) != cudaSuccess)
     return 0;
   return n;
 }
 
-template <int D, int NCW, int NSTAGE>
+template <int D, int NCW, int NSTAGE, int N8>
 cudaError_t launch_mma_t(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
                          dim3 grid, size_t smem, cudaStream_t stream) {
-  auto kern = pa_partition_mma_kernel<D, NCW, NSTAGE>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kern = pa_partition_mma_kernel<D, NCW, NSTAGE, N8>;
+  cudaError_t e = ensure_smem_attrs(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   kern<<<grid, 32 * (NCW + 1), smem, stream>>>(a, tk, tv);
   return cudaGetLastError();
 }
 
-template <int D, int NCW, int NSTAGE>
+template <int D, int NCW, int NSTAGE, int N8>
 int occupancy_mma_t(size_t smem) {
-  auto kern = pa_partition_mma_kernel<D, NCW, NSTAGE>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-      cudaSuccess)
-    return 0;
+  auto kern = pa_partition_mma_kernel<D, NCW, NSTAGE, N8>;
+  if (ensure_smem_attrs(reinterpret_cast<const void*>(kern), smem) != cudaSuccess) return 0;
   int n = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 32 * (NCW + 1), smem) != cudaSuccess)
     return 0;
@@ -943,21 +1051,27 @@ size_t mma_smem_bytes(int head_dim, int stages, int part_tokens, int block_size)
   return 1024 + ring + 2 * (size_t)stages * sizeof(uint64_t) + nbt * sizeof(int);
 }
 
-#define PA_MMA_DISPATCH(CALL)                                                       \
-  if (k.head_dim == 128 && k.consumer_warps == 4 && k.stages == 3) CALL(128, 4, 3); \
-  if (k.head_dim == 64 && k.consumer_warps == 4 && k.stages == 4) CALL(64, 4, 4);
+#define PA_MMA_DISPATCH(CALL)                                            \
+  if (k.head_dim == 128 && k.consumer_warps == 4 && k.stages == 3 && k.n8 == 1) \
+    CALL(128, 4, 3, 1);                                                  \
+  if (k.head_dim == 128 && k.consumer_warps == 4 && k.stages == 3 && k.n8 == 2) \
+    CALL(128, 4, 3, 2);                                                  \
+  if (k.head_dim == 64 && k.consumer_warps == 4 && k.stages == 4 && k.n8 == 1)  \
+    CALL(64, 4, 4, 1);                                                   \
+  if (k.head_dim == 64 && k.consumer_warps == 4 && k.stages == 4 && k.n8 == 2)  \
+    CALL(64, 4, 4, 2);
 
 cudaError_t launch_partition_mma(const DecodeArgs& a, const KernelShape& k, const CUtensorMap& tk,
                                  const CUtensorMap& tv, dim3 grid, size_t smem,
                                  cudaStream_t stream) {
-#define PA_CALL(D, N, S) return launch_mma_t<D, N, S>(a, tk, tv, grid, smem, stream)
+#define PA_CALL(D, N, S, N8) return launch_mma_t<D, N, S, N8>(a, tk, tv, grid, smem, stream)
   PA_MMA_DISPATCH(PA_CALL)
 #undef PA_CALL
   return cudaErrorInvalidValue;
 }
 
 int occupancy_partition_mma(const KernelShape& k, size_t smem) {
-#define PA_CALL(D, N, S) return occupancy_mma_t<D, N, S>(smem)
+#define PA_CALL(D, N, S, N8) return occupancy_mma_t<D, N, S, N8>(smem)
   PA_MMA_DISPATCH(PA_CALL)
 #undef PA_CALL
   return 0;
@@ -991,14 +1105,28 @@ int occupancy_partition_fma(const KernelShape& k, size_t smem) {
 }
 
 cudaError_t launch_reduce(const DecodeArgs& a, cudaStream_t stream) {
-  const dim3 grid(a.max_rows, a.num_kv_heads, a.batch);
-  if (a.head_dim == 128)
-    pa_reduce_kernel<128><<<grid, 256, 0, stream>>>(a);
-  else if (a.head_dim == 64)
-    pa_reduce_kernel<64><<<grid, 256, 0, stream>>>(a);
-  else
-    return cudaErrorInvalidValue;
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.max_rows, a.num_kv_heads, a.batch);
+  // about eight partitions per warp, 1 to 16 warps
+  const int nw = max(1, min(16, (a.max_parts + 7) / 8));
+  cfg.blockDim = dim3(32 * nw);
+  cfg.dynamicSmemBytes = (size_t)a.max_parts * sizeof(float);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const void* kern = a.head_dim == 128 ? reinterpret_cast<const void*>(pa_reduce_kernel<128>)
+                                        : reinterpret_cast<const void*>(pa_reduce_kernel<64>);
+  if (a.head_dim != 128 && a.head_dim != 64) return cudaErrorInvalidValue;
+  if (cfg.dynamicSmemBytes > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)cfg.dynamicSmemBytes);
+    if (e != cudaSuccess) return e;
+  }
+  if (a.head_dim == 128) return cudaLaunchKernelEx(&cfg, pa_reduce_kernel<128>, a);
+  return cudaLaunchKernelEx(&cfg, pa_reduce_kernel<64>, a);
 }
 
 cudaError_t launch_ranges(int32_t* lo, int32_t* hi, const int32_t* seq_lens,

@@ -41,6 +41,7 @@ struct KernelShape {
   int head_dim;
   int consumer_warps;
   int stages;
+  int n8;  // tensor-core variant: 8-row n-tiles per compute warp (1 or 2)
 };
 
 // Dynamic shared memory of the FMA partition kernel.

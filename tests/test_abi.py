@@ -165,21 +165,24 @@ def test_plan_row_slabs_for_many_rows():
     assert fma.max_rows == 32 and fma.slab_rows == 32 and fma.grid_y == 8
     kw.update(num_kv_heads=4, max_query_len_hint=5, batch=2)
     big = plan(**kw)
-    assert big.max_rows == 80 and big.grid_y == 4 * 2
+    assert big.max_rows == 80 and big.slab_rows == 64 and big.grid_y == 4 * 2
     big_fma = plan(force_variant=pa.PA_VARIANT_FMA, **kw)
     assert big_fma.grid_y == 4 * 3
 
 
-def test_plan_variant_follows_row_density():
-    # group x queryLen rows: 4 -> CUDA-core FMA, 8 and more -> tensor-core tiles
+def test_plan_variant_and_tile_width():
+    # tensor-core kernel by default; one 8-row n-tile per warp up to 8 rows, two above
     sparse = plan(batch=32, num_q_heads=32, num_kv_heads=8, head_dim=128, num_blocks=20000,
                   max_blocks_per_seq=512, max_span_hint=8192)
     dense = plan(batch=1, num_q_heads=8, num_kv_heads=1, head_dim=128, num_blocks=8193,
                  max_blocks_per_seq=8192, max_span_hint=131072)
-    mtp = plan(batch=2, num_q_heads=8, num_kv_heads=4, head_dim=64, num_blocks=100,
+    mtp = plan(batch=2, num_q_heads=16, num_kv_heads=4, head_dim=64, num_blocks=100,
                max_blocks_per_seq=50, max_span_hint=700, max_query_len_hint=4)
-    assert sparse.variant == pa.PA_VARIANT_FMA
-    assert dense.variant == pa.PA_VARIANT_MMA and mtp.variant == pa.PA_VARIANT_MMA
+    assert sparse.variant == dense.variant == mtp.variant == pa.PA_VARIANT_MMA
+    assert sparse.slab_rows == dense.slab_rows == 32 and mtp.slab_rows == 64
+    fma = plan(batch=32, num_q_heads=32, num_kv_heads=8, head_dim=128, num_blocks=20000,
+               max_blocks_per_seq=512, max_span_hint=8192, force_variant=pa.PA_VARIANT_FMA)
+    assert fma.variant == pa.PA_VARIANT_FMA and fma.slab_rows == 16
     forced = plan(batch=1, num_q_heads=8, num_kv_heads=1, head_dim=128, num_blocks=8193,
                   max_blocks_per_seq=8192, max_span_hint=131072, force_variant=pa.PA_VARIANT_FMA)
     assert forced.variant == pa.PA_VARIANT_FMA

@@ -78,12 +78,10 @@ def test_scaled_named_workloads(cfg, parts, variant):
     check_full(wl, out, f"scaled cfg{cfg} parts={parts} variant={variant}")
 
 
-def test_dispatcher_picks_fma_for_sparse_rows_and_mma_for_dense_tiles():
-    _, p2 = pa.pa_plan(pa.params_for(dev(scaled(2))), 16)
-    _, p4 = pa.pa_plan(pa.params_for(dev(scaled(4))), 16)
-    _, p5 = pa.pa_plan(pa.params_for(dev(scaled(5))), 1024)
-    assert p2.variant == pa.PA_VARIANT_FMA
-    assert p4.variant == pa.PA_VARIANT_MMA and p5.variant == pa.PA_VARIANT_MMA
+def test_dispatcher_defaults_to_the_tensor_core_kernel():
+    for cfg, bs in ((2, 16), (4, 16), (5, 1024)):
+        _, info = pa.pa_plan(pa.params_for(dev(scaled(cfg))), bs)
+        assert info.variant == pa.PA_VARIANT_MMA
 
 
 @pytest.mark.parametrize("variant", [pa.PA_VARIANT_FMA, pa.PA_VARIANT_MMA])
