@@ -147,7 +147,8 @@ int pa_decode(void *dst, const void *q, const void *kCache, const void *vCache,
  * zero span hint it assumes the longest row fills max_blocks_per_seq blocks,
  * with a zero query-length hint it assumes one query token per row (size the
  * workspace from real hints when rows carry several query tokens).
- * Returns 0 when the call is one-shot; (size_t)-1 on invalid params.
+ * Returns 0 when the call is one-shot; (size_t)-1 on invalid params.  The
+ * workspace needs no initialisation.
  * Host only; needs a CUDA device only when num_sms is not fixed (it queries
  * the current device's SM count and occupancy).
  */

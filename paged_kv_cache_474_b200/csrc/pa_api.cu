@@ -9,7 +9,8 @@
 // the SM count.  Here the partition size comes from the longest windowed span,
 // the number of (row, kv head) units and the SMs x resident CTAs of the
 // chosen kernel: few units get one balanced wave of partitions, many units
-// get about four waves so ragged rows even out.  One partition per row means
+// get partitions of 2048..4096 tokens (about four waves where that fits).
+// One partition per row means
 // the one-shot path: the kernel writes dst itself, with no workspace and no
 // reduce (aiter PR #2914 "Pa gluon swa mtp opt", one_shot).
 #include <algorithm>
@@ -49,6 +50,8 @@ int succeed() {
 
 constexpr int TS = pa::kStageTokens;
 constexpr int kMinPartTokens = 256;
+constexpr int kManyUnitsMinTokens = 2048;
+constexpr int kManyUnitsMaxTokens = 4096;
 
 bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
@@ -193,10 +196,18 @@ int make_plan(const pa_params* p, int bs, int span, int qlen, int num_sms, int c
   if (p->force_partitions > 0) {
     ptok = cdiv(cdiv(span, p->force_partitions), TS) * TS;
   } else {
-    const long long waves = (units * 4 <= slots) ? 1 : 4;
-    const long long want = std::max<long long>(1, cdiv(waves * slots, std::max<long long>(units, 1)));
-    ptok = cdiv(cdiv(span, want), TS) * TS;
-    ptok = std::max<long long>(ptok, kMinPartTokens);
+    if (units * 4 <= slots) {
+      // few units: one balanced wave over every resident-CTA slot
+      const long long want = std::max<long long>(1, cdiv(slots, std::max<long long>(units, 1)));
+      ptok = std::max<long long>(cdiv(cdiv(span, want), TS) * TS, kMinPartTokens);
+    } else {
+      // many units: about four waves, but partitions of 2048..4096 tokens,
+      // long enough to amortise a CTA's start-up and short enough that
+      // ragged rows even out (measured on the named workloads)
+      const long long want = std::max<long long>(1, cdiv(4 * slots, units));
+      ptok = cdiv(cdiv(span, want), TS) * TS;
+      ptok = std::min<long long>(std::max<long long>(ptok, kManyUnitsMinTokens), kManyUnitsMaxTokens);
+    }
   }
   ptok = std::min<long long>(std::max<long long>(ptok, TS), cap);
   // The reduce keeps one weight per partition in smem: at most 16384.
@@ -353,8 +364,9 @@ int decode_impl(void* dst, const void* q, const void* kCache, const void* vCache
   a.windows = p->windows;
   a.dst = static_cast<__nv_bfloat16*>(dst);
   if (!in.one_shot) {
-    a.ws_lse = static_cast<float*>(p->workspace);
-    a.ws_o = reinterpret_cast<float*>(static_cast<char*>(p->workspace) + pl.lse_bytes);
+    char* ws = static_cast<char*>(p->workspace);
+    a.ws_lse = reinterpret_cast<float*>(ws);
+    a.ws_o = reinterpret_cast<float*>(ws + pl.lse_bytes);
   }
   a.scale_log2 = scale * 1.4426950408889634f;
   a.window = window;

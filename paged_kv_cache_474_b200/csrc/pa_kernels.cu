@@ -473,9 +473,35 @@ __global__ void __maxnreg__(N8 == 1 ? 128 : 168)
   const int slab = blockIdx.y / a.num_kv_heads;
   const int part = blockIdx.x;
 
+  __shared__ int s_qoff;
+
+  // Nothing here depends on the inputs: set up the pipeline while the
+  // previous kernel on the stream may still be finishing (this kernel is
+  // launched with programmatic stream serialization), then wait for it.
+  if (threadIdx.x == 0) {
+    prefetch_tensormap(&tmk);
+    prefetch_tensormap(&tmv);
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(smem_u32(&bars[s]), 1);              // full: copy-warp arrival + tx bytes
+      mbar_init(smem_u32(&bars[NSTAGE + s]), NCW);   // empty: one arrival per compute warp
+    }
+    fence_mbar_init();
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
   const int S = a.seq_lens[b];
   const int L = a.query_lens[b];
   const int w = a.windows ? a.windows[b] : a.window;
+  // A row without a window starts its partitions at token 0, so the copy warp
+  // can fetch the partition's block-table slice while the lengths are still
+  // in flight (entries past the row's last block are read but never used).
+  const bool spec_table = (a.windows == nullptr && a.window == 0);
+  if (warp == 0 && spec_table) {
+    const int sj0 = (part * a.part_tokens) >> a.block_shift;
+    const int sn = min(a.part_tokens / a.block_size + 2, a.max_blocks_per_seq - sj0);
+    for (int i = lane; i < sn; i += 32)
+      bt_s[i] = a.block_tables[(size_t)b * a.max_blocks_per_seq + sj0 + i];
+  }
   if (L <= 0) return;
   const bool lead = (part == 0 && slab == 0 && kvh == 0 && threadIdx.x == 0);
   if (L > S || w < 0 || S > a.max_blocks_per_seq * a.block_size) {
@@ -499,15 +525,6 @@ __global__ void __maxnreg__(N8 == 1 ? 128 : 168)
   const int jb0 = p0 >> a.block_shift;
   const int nbt = ((p1 - 1) >> a.block_shift) - jb0 + 1;
 
-  if (threadIdx.x == 0) {
-    prefetch_tensormap(&tmk);
-    prefetch_tensormap(&tmv);
-    for (int s = 0; s < NSTAGE; ++s) {
-      mbar_init(smem_u32(&bars[s]), 1);
-      mbar_init(smem_u32(&bars[NSTAGE + s]), NCW);
-    }
-    fence_mbar_init();
-  }
   __syncthreads();
   // Let the reduce grid launch now; it waits for this grid's completion
   // before reading any partial.
@@ -526,9 +543,10 @@ __global__ void __maxnreg__(N8 == 1 ? 128 : 168)
   if (warp == 0) {
     // ------------------------------ copy warp ------------------------------
     // This warp alone reads the partition's block-table slice, so the first
-    // copies go out without waiting for the compute warps' prologue.
+    // copies go out without waiting for the compute warps' prologue.  (With
+    // spec_table the slice is already in smem: same start, same lanes.)
     for (int i = lane; i < nbt; i += 32) {
-      int phys = a.block_tables[(size_t)b * a.max_blocks_per_seq + jb0 + i];
+      int phys = spec_table ? bt_s[i] : a.block_tables[(size_t)b * a.max_blocks_per_seq + jb0 + i];
       if (phys < 0 || phys >= a.num_blocks) {
         atomicOr(&g_pa_status, PA_DEV_BAD_BLOCK);
         phys = -1;
@@ -579,7 +597,6 @@ __global__ void __maxnreg__(N8 == 1 ? 128 : 168)
         mbar_wait(smem_u32(&bars[k % NSTAGE]), (k / NSTAGE) & 1);
     }
     __syncwarp();
-    qoff = row_token_offset(a.query_lens, b, lane);
   } else {
     // ----------------------------- compute warps ---------------------------
     const int cw = warp - 1;
@@ -588,6 +605,7 @@ __global__ void __maxnreg__(N8 == 1 ? 128 : 168)
     const int nslice = (NCW - 1 - rt) / NRT + 1;
     const int quad = lane >> 2, qi = lane & 3;
     qoff = row_token_offset(a.query_lens, b, lane);
+    if (warp == 1 && lane == 0) s_qoff = qoff;  // for the copy warp's share of the merge
     const int brs = a.block_shift < 6 ? a.block_shift : 6;  // log2(BR)
     // lane parts of the ldmatrix row addresses (token row within the chunk,
     // 16-byte chunk parity) for K (A operand) and V (A operand, transposed)
@@ -764,6 +782,7 @@ __global__ void __maxnreg__(N8 == 1 ? 128 : 168)
       }
   }
   __syncthreads();
+  if (warp == 0) qoff = s_qoff;
 
   // ----------------- merge the compute warps' partials --------------------
   for (int idx = threadIdx.x; idx < Rs * D; idx += blockDim.x) {
@@ -1029,8 +1048,20 @@ cudaError_t launch_mma_t(const DecodeArgs& a, const CUtensorMap& tk, const CUten
   auto kern = pa_partition_mma_kernel<D, NCW, NSTAGE, N8>;
   cudaError_t e = ensure_smem_attrs(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, 32 * (NCW + 1), smem, stream>>>(a, tk, tv);
-  return cudaGetLastError();
+  // Programmatic stream serialization: CTAs may start (and set up their
+  // pipeline) while the previous kernel drains; they wait on griddepcontrol
+  // before reading any input.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(32 * (NCW + 1));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a, tk, tv);
 }
 
 template <int D, int NCW, int NSTAGE, int N8>
