@@ -205,8 +205,13 @@ int make_plan(const pa_params* p, int bs, int span, int qlen, int num_sms, int c
       // long enough to amortise a CTA's start-up and short enough that
       // ragged rows even out (measured on the named workloads)
       const long long want = std::max<long long>(1, cdiv(4 * slots, units));
-      ptok = cdiv(cdiv(span, want), TS) * TS;
-      ptok = std::min<long long>(std::max<long long>(ptok, kManyUnitsMinTokens), kManyUnitsMaxTokens);
+      const long long target = std::min<long long>(
+          std::max<long long>(cdiv(span, want), kManyUnitsMinTokens), kManyUnitsMaxTokens);
+      // equal partitions: round the count to the nearest, so a row just over
+      // a multiple of the target does not end in a sliver partition
+      const long long aligned_span = (long long)span + TS - 1;
+      const long long np = std::max<long long>(1, (aligned_span + target / 2) / target);
+      ptok = cdiv(cdiv(aligned_span, np), TS) * TS;
     }
   }
   ptok = std::min<long long>(std::max<long long>(ptok, TS), cap);

@@ -429,7 +429,8 @@ struct MmaTraits {
 template <int D, int NCW, int N8>
 struct MmaCombine {
   static constexpr int RT = 8 * N8;  // rows per warp tile
-  static constexpr int ACC_FLOATS = NCW * RT * D;
+  static constexpr int LD = D + 4;   // padded row stride: conflict-free fragment stores
+  static constexpr int ACC_FLOATS = NCW * RT * LD;
   static constexpr int L_FLOATS = NCW * RT;
   static constexpr int M_FLOATS = NCW * RT;
   static constexpr int BYTES = (ACC_FLOATS + L_FLOATS + M_FLOATS) * 4;
@@ -474,6 +475,7 @@ __global__ void __maxnreg__(N8 == 1 ? 128 : 168)
   const int part = blockIdx.x;
 
   __shared__ int s_qoff;
+  __shared__ float s_fac[NCW][64], s_rowm[64], s_rowz[64];  // warp-merge factors (rows <= 64)
 
   // Nothing here depends on the inputs: set up the pipeline while the
   // previous kernel on the stream may still be finishing (this kernel is
@@ -765,7 +767,7 @@ __global__ void __maxnreg__(N8 == 1 ? 128 : 168)
       for (int n = 0; n < N8; ++n)
 #pragma unroll
         for (int e = 0; e < 4; ++e)
-          comb_acc[(cw * RT + n * 8 + 2 * qi + (e & 1)) * D + md * 16 + quad + ((e >> 1) << 3)] =
+          comb_acc[(cw * RT + n * 8 + 2 * qi + (e & 1)) * C::LD + md * 16 + quad + ((e >> 1) << 3)] =
               o[md][n][e];
 #pragma unroll
     for (int n = 0; n < N8; ++n)
@@ -785,30 +787,51 @@ __global__ void __maxnreg__(N8 == 1 ? 128 : 168)
   if (warp == 0) qoff = s_qoff;
 
   // ----------------- merge the compute warps' partials --------------------
-  for (int idx = threadIdx.x; idx < Rs * D; idx += blockDim.x) {
-    const int rloc = idx / D;
-    const int d = idx - rloc * D;
-    const int rti = rloc / RT, rr8 = rloc - rti * RT;
+  // Per row: the slices' common max M, each slice's factor 2^(m_c - M) and
+  // the sum Z; then every float4 column is an independent weighted sum.
+  for (int r = threadIdx.x; r < Rs; r += blockDim.x) {
+    const int rti = r / RT, rr8 = r - (r / RT) * RT;
     float M = kNegInf;
     for (int c = rti; c < NCW; c += NRT) M = fmaxf(M, comb_m[c * RT + rr8]);
-    float Z = 0.f, O = 0.f;
-    if (M != kNegInf) {
-      for (int c = rti; c < NCW; c += NRT) {
-        const float sc = ex2(comb_m[c * RT + rr8] - M);
-        Z += sc * comb_l[c * RT + rr8];
-        O += sc * comb_acc[(c * RT + rr8) * D + d];
-      }
+    float Z = 0.f;
+    for (int c = rti; c < NCW; c += NRT) {
+      const float f = (M == kNegInf) ? 0.f : ex2(comb_m[c * RT + rr8] - M);
+      s_fac[c][r] = f;
+      Z += f * comb_l[c * RT + rr8];
     }
-    const int rr = row0 + rloc;
+    s_rowm[r] = M;
+    s_rowz[r] = Z;
+  }
+  __syncthreads();
+  constexpr int C4 = D / 4;
+  for (int it = threadIdx.x; it < Rs * C4; it += blockDim.x) {
+    const int r = it / C4, c4 = it - (it / C4) * C4;
+    const int rti = r / RT, rr8 = r - (r / RT) * RT;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c = rti; c < NCW; c += NRT) {
+      const float f = s_fac[c][r];
+      const float4 v = *reinterpret_cast<const float4*>(comb_acc + (c * RT + rr8) * C::LD + c4 * 4);
+      acc.x += f * v.x;
+      acc.y += f * v.y;
+      acc.z += f * v.z;
+      acc.w += f * v.w;
+    }
+    const float Z = s_rowz[r];
+    const int rr = row0 + r;
     if (nparts == 1) {
+      const float inv = 1.f / Z;
       const int i = rr / a.group, j = rr - (rr / a.group) * a.group;
-      a.dst[((size_t)(qoff + i) * a.num_q_heads + (size_t)kvh * a.group + j) * D + d] =
-          __float2bfloat16_rn(O / Z);
+      __nv_bfloat16* dp =
+          a.dst + ((size_t)(qoff + i) * a.num_q_heads + (size_t)kvh * a.group + j) * D + c4 * 4;
+      *reinterpret_cast<__nv_bfloat162*>(dp) = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+      *reinterpret_cast<__nv_bfloat162*>(dp + 2) = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
     } else {
+      const float inv = Z > 0.f ? 1.f / Z : 0.f;
       const size_t base =
           ((size_t)(b * a.num_kv_heads + kvh) * a.max_parts + part) * a.max_rows + rr;
-      a.ws_o[base * D + d] = Z > 0.f ? O / Z : 0.f;
-      if (d == 0) a.ws_lse[base] = Z > 0.f ? M + lg2(Z) : kNegInf;
+      *reinterpret_cast<float4*>(a.ws_o + base * D + c4 * 4) =
+          make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+      if (c4 == 0) a.ws_lse[base] = Z > 0.f ? s_rowm[r] + lg2(Z) : kNegInf;
     }
   }
 }
@@ -819,25 +842,30 @@ __global__ void __maxnreg__(N8 == 1 ? 128 : 168)
 // dst = sum_p w_p O_p / sum_p w_p.  Partials are normalised, so the weights
 // carry each partition's softmax mass.
 //
-// One CTA per (row, kv head, batch row).  The CTA first loads every lse_p
-// (one coalesced pass), forms the weights in smem, then its warps sum w_p O_p
-// over interleaved partitions with four independent partial loads in flight
-// per lane, each lane owning D/32 consecutive dims; warps merge through smem.
-// Launched with programmatic stream serialization: it may be scheduled while
-// the partition kernel drains and waits on griddepcontrol before reading.
+// One CTA per (row, kv head, batch row) and DSPLIT-th of head_dim.  The CTA
+// loads every lse_p once (coalesced), keeps the weights in smem, then its
+// warps sum w_p O_p: a partial's slice is DC/4 float4, so a warp reads
+// 32/(DC/4) partials per load and keeps BATCH loads in flight per lane.
+// Rows with hundreds of partials split head_dim over several CTAs so more SMs
+// pull partials from L2.  Launched with programmatic stream serialization: it
+// may be scheduled while the partition kernel drains and waits on
+// griddepcontrol before reading.
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, int DSPLIT>
 __global__ void __launch_bounds__(512) pa_reduce_kernel(const __grid_constant__ DecodeArgs a) {
-  constexpr int VPL = D / 32;  // dims per lane
-  constexpr int BATCH = 4;     // partial loads in flight per lane
+  constexpr int DC = D / DSPLIT;  // dims per CTA
+  constexpr int LPP = DC / 4;     // lanes per partial slice (one float4 each)
+  constexpr int PPW = 32 / LPP;   // partials per warp load
+  constexpr int BATCH = 8;        // loads in flight per lane
   extern __shared__ float s_w[];  // [max_parts] weights
   __shared__ float s_red[16];
-  __shared__ __align__(16) float s_acc[16][D];
+  __shared__ float4 s_acc[16][LPP];
   __shared__ float s_M, s_Z;
   __shared__ int s_qoff;
 
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int rr = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int rr = blockIdx.x / DSPLIT, ch = blockIdx.x - (blockIdx.x / DSPLIT) * DSPLIT;
+  const int kvh = blockIdx.y, b = blockIdx.z;
   const int S = a.seq_lens[b];
   const int L = a.query_lens[b];
   const int w = a.windows ? a.windows[b] : a.window;
@@ -891,54 +919,54 @@ __global__ void __launch_bounds__(512) pa_reduce_kernel(const __grid_constant__ 
     s_Z = x;
   }
 
-  float acc[VPL];
-#pragma unroll
-  for (int v = 0; v < VPL; ++v) acc[v] = 0.f;
-  const float* obase = a.ws_o + (ubase * a.max_rows + rr) * D + lane * VPL;
-  const size_t pstride = (size_t)a.max_rows * D;
-  for (int p0 = warp; p0 < nparts; p0 += BATCH * nw) {
-    float o[BATCH][VPL];
+  const int sub = lane / LPP, c4 = lane - (lane / LPP) * LPP;
+  const float4* ob =
+      reinterpret_cast<const float4*>(a.ws_o + (ubase * a.max_rows + rr) * D + ch * DC) + c4;
+  const size_t pst4 = (size_t)a.max_rows * D / 4;  // float4 stride between partials
+  const int step = nw * PPW;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int p0 = warp * PPW + sub; p0 < nparts; p0 += BATCH * step) {
+    float4 o[BATCH];
 #pragma unroll
     for (int u = 0; u < BATCH; ++u) {
-      const int p = p0 + u * nw;
-      if (p < nparts) {
-        if constexpr (VPL == 4) {
-          const float4 t = *reinterpret_cast<const float4*>(obase + p * pstride);
-          o[u][0] = t.x, o[u][1] = t.y, o[u][2] = t.z, o[u][3] = t.w;
-        } else {
-          const float2 t = *reinterpret_cast<const float2*>(obase + p * pstride);
-          o[u][0] = t.x, o[u][1] = t.y;
-        }
-      } else {
-#pragma unroll
-        for (int v = 0; v < VPL; ++v) o[u][v] = 0.f;
-      }
+      const int p = p0 + u * step;
+      o[u] = p < nparts ? ob[(size_t)p * pst4] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
     for (int u = 0; u < BATCH; ++u) {
-      const int p = p0 + u * nw;
+      const int p = p0 + u * step;
       const float wt = p < nparts ? s_w[p] : 0.f;
-#pragma unroll
-      for (int v = 0; v < VPL; ++v) acc[v] += wt * o[u][v];
+      acc.x += wt * o[u].x;
+      acc.y += wt * o[u].y;
+      acc.z += wt * o[u].z;
+      acc.w += wt * o[u].w;
     }
   }
 #pragma unroll
-  for (int v = 0; v < VPL; ++v) s_acc[warp][lane * VPL + v] = acc[v];
+  for (int off = LPP; off < 32; off <<= 1) {
+    acc.x += __shfl_xor_sync(FULL, acc.x, off);
+    acc.y += __shfl_xor_sync(FULL, acc.y, off);
+    acc.z += __shfl_xor_sync(FULL, acc.z, off);
+    acc.w += __shfl_xor_sync(FULL, acc.w, off);
+  }
+  if (sub == 0) s_acc[warp][c4] = acc;
   __syncthreads();
-  if (warp == 0) {
-    float out[VPL];
-#pragma unroll
-    for (int v = 0; v < VPL; ++v) out[v] = 0.f;
-    for (int i = 0; i < nw; ++i)
-#pragma unroll
-      for (int v = 0; v < VPL; ++v) out[v] += s_acc[i][lane * VPL + v];
+  if (warp == 0 && lane < LPP) {
+    float4 out = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i = 0; i < nw; ++i) {
+      const float4 v = s_acc[i][lane];
+      out.x += v.x;
+      out.y += v.y;
+      out.z += v.z;
+      out.w += v.w;
+    }
     const float inv = 1.f / s_Z;
     const int i = rr / a.group, j = rr - (rr / a.group) * a.group;
-    __nv_bfloat16* dp = a.dst + ((size_t)(s_qoff + i) * a.num_q_heads + (size_t)kvh * a.group + j) * D +
-                        lane * VPL;
-#pragma unroll
-    for (int v = 0; v < VPL; v += 2)
-      *reinterpret_cast<__nv_bfloat162*>(dp + v) = __floats2bfloat162_rn(out[v] * inv, out[v + 1] * inv);
+    __nv_bfloat16* dp = a.dst +
+                        ((size_t)(s_qoff + i) * a.num_q_heads + (size_t)kvh * a.group + j) * D +
+                        ch * DC + lane * 4;
+    *reinterpret_cast<__nv_bfloat162*>(dp) = __floats2bfloat162_rn(out.x * inv, out.y * inv);
+    *reinterpret_cast<__nv_bfloat162*>(dp + 2) = __floats2bfloat162_rn(out.z * inv, out.w * inv);
   }
 }
 
@@ -1135,11 +1163,13 @@ int occupancy_partition_fma(const KernelShape& k, size_t smem) {
   return 0;
 }
 
-cudaError_t launch_reduce(const DecodeArgs& a, cudaStream_t stream) {
+template <int D, int DSPLIT>
+cudaError_t launch_reduce_t(const DecodeArgs& a, cudaStream_t stream) {
+  constexpr int PPW = 32 / (D / DSPLIT / 4);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.max_rows, a.num_kv_heads, a.batch);
-  // about eight partitions per warp, 1 to 16 warps
-  const int nw = max(1, min(16, (a.max_parts + 7) / 8));
+  cfg.gridDim = dim3(a.max_rows * DSPLIT, a.num_kv_heads, a.batch);
+  // warps so that each lane has about one batch of eight loads, 1 to 16
+  const int nw = max(1, min(16, (a.max_parts + PPW * 8 - 1) / (PPW * 8)));
   cfg.blockDim = dim3(32 * nw);
   cfg.dynamicSmemBytes = (size_t)a.max_parts * sizeof(float);
   cfg.stream = stream;
@@ -1148,16 +1178,23 @@ cudaError_t launch_reduce(const DecodeArgs& a, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const void* kern = a.head_dim == 128 ? reinterpret_cast<const void*>(pa_reduce_kernel<128>)
-                                        : reinterpret_cast<const void*>(pa_reduce_kernel<64>);
-  if (a.head_dim != 128 && a.head_dim != 64) return cudaErrorInvalidValue;
+  auto kern = pa_reduce_kernel<D, DSPLIT>;
   if (cfg.dynamicSmemBytes > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)cfg.dynamicSmemBytes);
     if (e != cudaSuccess) return e;
   }
-  if (a.head_dim == 128) return cudaLaunchKernelEx(&cfg, pa_reduce_kernel<128>, a);
-  return cudaLaunchKernelEx(&cfg, pa_reduce_kernel<64>, a);
+  return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+cudaError_t launch_reduce(const DecodeArgs& a, cudaStream_t stream) {
+  // Rows with many partials split head_dim over several CTAs (32 dims each).
+  const bool split = a.max_parts >= 64;
+  if (a.head_dim == 128)
+    return split ? launch_reduce_t<128, 4>(a, stream) : launch_reduce_t<128, 1>(a, stream);
+  if (a.head_dim == 64)
+    return split ? launch_reduce_t<64, 2>(a, stream) : launch_reduce_t<64, 1>(a, stream);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_ranges(int32_t* lo, int32_t* hi, const int32_t* seq_lens,

@@ -84,11 +84,13 @@ def test_dispatcher_defaults_to_the_tensor_core_kernel():
         assert info.variant == pa.PA_VARIANT_MMA
 
 
+@pytest.mark.parametrize("head_dim", [64, 128])
 @pytest.mark.parametrize("variant", [pa.PA_VARIANT_FMA, pa.PA_VARIANT_MMA])
 @pytest.mark.parametrize("parts", [1, 2, 3, 7, 64, 200])
-def test_split_k_invariance(parts, variant):
+def test_split_k_invariance(parts, variant, head_dim):
+    # 64 and 200 partitions also exercise the reduce that splits head_dim over CTAs
     wl = make_workload(seq_lens=[5000, 3333, 77], query_lens=[1, 3, 2], num_q_heads=8,
-                       num_kv_heads=2, head_dim=128, block_size=16, window=0, seed=7)
+                       num_kv_heads=2, head_dim=head_dim, block_size=16, window=0, seed=7)
     d = dev(wl)
     out = pa.decode(d, force_partitions=parts, force_variant=variant)
     check_full(wl, out, f"parts={parts}")
