@@ -141,7 +141,7 @@ class ClockSampler:
 def traffic_from_profiles(kernel_src_hash: str, workload: str):
     """DRAM bytes per launch of the partition kernel from the committed ncu
     summary, if it was taken on the current kernel source and this workload."""
-    path = os.path.join(ROOT, "profiles", "partition_traffic.json")
+    path = os.path.join(ROOT, "profiles", "partition_traffic.txt")
     try:
         with open(path) as f:
             d = json.load(f)
@@ -399,7 +399,7 @@ def run_other_configs(args, local_rank):
         # (one per layer of a model, >= 4x L2 in total), so no call finds its
         # KV in L2 and each call's launch overlaps the previous call's tail.
         pool = wl.k_cache.numel() * wl.k_cache.element_size() * 2
-        nlay = max(1, -(-(4 * l2) // pool))
+        nlay = max(1, min(64, -(-(4 * l2) // pool)))
         layers = [(wl.k_cache, wl.v_cache)] + [(wl.k_cache.clone(), wl.v_cache.clone())
                                                for _ in range(nlay - 1)]
         def layer_call(i):
