@@ -431,6 +431,36 @@ def run_other_configs(args, local_rank):
                                   "partition_tokens": info.partition_tokens}
         del wl, ws, out, layers
         torch.cuda.empty_cache()
+    # The ExecuTorch page's standalone kernel benchmark shape (B=1, H_q=16,
+    # H_kv=2, D=256, one decode token) over a paged cache, per context length.
+    from paged_kv_cache_474_b200.workloads import make_workload
+    sweep = {}
+    for lk in (64, 512, 4096, 8192, 16384):
+        wl = make_workload(seq_lens=[lk], query_lens=[1], num_q_heads=16, num_kv_heads=2,
+                           head_dim=256, block_size=16, seed=lk, device=device)
+        kv, qo = algorithmic_bytes(wl)
+        p = pa.params_for(wl)
+        ws = pa.alloc_workspace(p, wl.block_size, device=device)
+        if ws is not None:
+            p.workspace, p.workspace_bytes = ws.data_ptr(), ws.numel()
+        out = torch.empty_like(wl.q)
+        c = (out.data_ptr(), wl.q.data_ptr(), wl.k_cache.data_ptr(), wl.v_cache.data_ptr(),
+             wl.block_tables.data_ptr(), wl.seq_lens.data_ptr(), wl.query_lens.data_ptr(),
+             wl.scale, wl.window, wl.block_size)
+        for _ in range(3):
+            pa.pa_decode(*c, p, sh)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(20)]
+        for a, b in ev:
+            flush_l2()
+            a.record(stream)
+            pa.pa_decode(*c, p, sh)
+            b.record(stream)
+        torch.cuda.synchronize()
+        us = statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3
+        sweep[str(lk)] = {"us_per_call": round(us, 2), "gbs": round((kv + qo) / us / 1e3, 1)}
+        del wl, ws, out
+    res["executorch_shape_B1_Hq16_Hkv2_D256"] = sweep
     if pa.pa_device_status(clear=True):
         raise RuntimeError("device status set during the per-config runs")
     return res

@@ -74,7 +74,7 @@ typedef struct pa_params {
     int batch;               /* rows */
     int num_q_heads;         /* H_q, a multiple of num_kv_heads */
     int num_kv_heads;        /* H_kv */
-    int head_dim;            /* 64 or 128 */
+    int head_dim;            /* 64, 128 or 256 (256: tensor-core variant) */
     int num_blocks;          /* KV pool size in blocks */
     int max_blocks_per_seq;  /* blockTables row stride (entries) */
     /* Host hints.  max_span_hint >= max_b union span, where a row's union
@@ -131,7 +131,7 @@ typedef struct pa_plan_info {
  *
  * All device pointers must be 16-byte aligned.  Returns PA_ERR_ARG for null
  * pointers, H_q % H_kv != 0, negative window or hints, misalignment;
- * PA_ERR_UNSUPPORTED for head_dim not in {64,128} or a block size outside
+ * PA_ERR_UNSUPPORTED for head_dim not in {64,128,256} or a block size outside
  * the set above; PA_ERR_WORKSPACE when split-K partials are needed and the
  * workspace is too small; PA_ERR_CUDA when a launch fails.
  */

@@ -94,8 +94,8 @@ int check_params(const pa_params* p, int bs) {
   if (p->num_q_heads % p->num_kv_heads != 0)
     return fail(PA_ERR_ARG, "H_q=%d is not a multiple of H_kv=%d", p->num_q_heads,
                 p->num_kv_heads);
-  if (p->head_dim != 64 && p->head_dim != 128)
-    return fail(PA_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", p->head_dim);
+  if (p->head_dim != 64 && p->head_dim != 128 && p->head_dim != 256)
+    return fail(PA_ERR_UNSUPPORTED, "head_dim %d not supported (64, 128 or 256)", p->head_dim);
   if (!is_pow2(bs) || bs < 16 || bs > 1024)
     return fail(PA_ERR_UNSUPPORTED, "kvBlockSize %d not supported (power of two in [16,1024])", bs);
   if (p->num_blocks <= 0 || p->max_blocks_per_seq <= 0)
@@ -162,17 +162,20 @@ int make_plan(const pa_params* p, int bs, int span, int qlen, int num_sms, int c
   if (variant == PA_VARIANT_AUTO) variant = rows_fit_tma ? PA_VARIANT_MMA : PA_VARIANT_FMA;
   if (variant == PA_VARIANT_MMA && !rows_fit_tma)
     return fail(PA_ERR_UNSUPPORTED, "KV pool rows exceed the tensor map's 32-bit coordinates");
+  if (variant == PA_VARIANT_FMA && p->head_dim == 256)
+    return fail(PA_ERR_UNSUPPORTED, "head_dim 256 runs on the tensor-core kernel only");
   const bool mma = variant == PA_VARIANT_MMA;
   const int ncw = mma ? 4 : (rmax <= 16 ? 4 : 8);
   // tensor-core warps cover 8 rows (one n-tile) when the unit has <= 8 rows,
-  // else 16; a CTA covers up to 4 such tiles.
-  const int n8 = (mma && rmax > 8) ? 2 : 1;
+  // else 16 (head_dim 256: always 8, its accumulators are twice as wide); a
+  // CTA covers up to 4 such tiles.
+  const int n8 = (mma && rmax > 8 && p->head_dim <= 128) ? 2 : 1;
   pl.shape.n8 = n8;
   const int slab_rows = mma ? 8 * n8 * ncw : 4 * ncw;
   const int nslab = (int)cdiv(rmax, slab_rows);
   pl.shape.head_dim = p->head_dim;
   pl.shape.consumer_warps = ncw;
-  pl.shape.stages = p->head_dim == 128 ? 3 : 4;
+  pl.shape.stages = p->head_dim == 64 ? 4 : 3;  // 16, 32 or 64 KB per stage
 
   // Partition-size cap: the CTA caches its slice of the block table in smem.
   const int cap = std::max(TS, ((pa::kMaxTableCache - 2) * bs) / TS * TS);

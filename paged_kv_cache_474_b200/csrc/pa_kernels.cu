@@ -450,9 +450,10 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
 }
 
 // Register caps keep 4 (one n-tile) or 3 (two n-tiles) warps per SM
-// sub-partition, so two CTAs fit per SM.
+// sub-partition, so two CTAs fit per SM; head_dim 256 runs one CTA per SM
+// (its 192 KB ring) and takes the larger cap for its wider accumulators.
 template <int D, int NCW, int NSTAGE, int N8>
-__global__ void __maxnreg__(N8 == 1 ? 128 : 168)
+__global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
     pa_partition_mma_kernel(const __grid_constant__ DecodeArgs a,
                             const __grid_constant__ CUtensorMap tmk,
                             const __grid_constant__ CUtensorMap tmv) {
@@ -1118,7 +1119,9 @@ size_t mma_smem_bytes(int head_dim, int stages, int part_tokens, int block_size)
   if (k.head_dim == 64 && k.consumer_warps == 4 && k.stages == 4 && k.n8 == 1)  \
     CALL(64, 4, 4, 1);                                                   \
   if (k.head_dim == 64 && k.consumer_warps == 4 && k.stages == 4 && k.n8 == 2)  \
-    CALL(64, 4, 4, 2);
+    CALL(64, 4, 4, 2);                                                   \
+  if (k.head_dim == 256 && k.consumer_warps == 4 && k.stages == 3 && k.n8 == 1) \
+    CALL(256, 4, 3, 1);
 
 cudaError_t launch_partition_mma(const DecodeArgs& a, const KernelShape& k, const CUtensorMap& tk,
                                  const CUtensorMap& tv, dim3 grid, size_t smem,
@@ -1188,12 +1191,15 @@ cudaError_t launch_reduce_t(const DecodeArgs& a, cudaStream_t stream) {
 }
 
 cudaError_t launch_reduce(const DecodeArgs& a, cudaStream_t stream) {
-  // Rows with many partials split head_dim over several CTAs (32 dims each).
+  // Rows with many partials split head_dim over several CTAs (32 dims each);
+  // a CTA covers at most 128 dims (one float4 per lane).
   const bool split = a.max_parts >= 64;
   if (a.head_dim == 128)
     return split ? launch_reduce_t<128, 4>(a, stream) : launch_reduce_t<128, 1>(a, stream);
   if (a.head_dim == 64)
     return split ? launch_reduce_t<64, 2>(a, stream) : launch_reduce_t<64, 1>(a, stream);
+  if (a.head_dim == 256)
+    return split ? launch_reduce_t<256, 8>(a, stream) : launch_reduce_t<256, 2>(a, stream);
   return cudaErrorInvalidValue;
 }
 

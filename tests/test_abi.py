@@ -54,7 +54,7 @@ def call(p, bs=16, window=0, scale=0.125, ptrs=16):
     (dict(num_q_heads=5), pa.PA_ERR_ARG),
     (dict(num_kv_heads=0), pa.PA_ERR_ARG),
     (dict(head_dim=96), pa.PA_ERR_UNSUPPORTED),
-    (dict(head_dim=256), pa.PA_ERR_UNSUPPORTED),
+    (dict(head_dim=512), pa.PA_ERR_UNSUPPORTED),
     (dict(batch=-1), pa.PA_ERR_ARG),
     (dict(num_blocks=0), pa.PA_ERR_ARG),
     (dict(max_span_hint=-3), pa.PA_ERR_ARG),
@@ -201,3 +201,13 @@ def test_plan_caps_partition_at_the_table_cache():
     info = plan(batch=1, num_q_heads=1, num_kv_heads=1, head_dim=64, num_blocks=70000,
                 max_blocks_per_seq=65536, max_span_hint=1 << 20, sms=1, occ=1)
     assert info.partition_tokens <= (1024 - 2) * 16
+
+
+def test_plan_head_dim_256_uses_the_tensor_core_kernel():
+    # the ExecuTorch page's H100 benchmark shape: B=1, H_q=16, H_kv=2, D=256
+    info = plan(batch=1, num_q_heads=16, num_kv_heads=2, head_dim=256, num_blocks=1100,
+                max_blocks_per_seq=1024, max_span_hint=16384, occ=1)
+    assert info.variant == pa.PA_VARIANT_MMA and info.slab_rows == 32
+    assert info.smem_bytes <= 227 * 1024
+    rc, _ = pa.pa_plan(base_params(head_dim=256, force_variant=pa.PA_VARIANT_FMA), 16, 148, 1)
+    assert rc == pa.PA_ERR_UNSUPPORTED

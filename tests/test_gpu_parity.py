@@ -334,3 +334,23 @@ def test_device_detects_rows_beyond_hints_and_bad_blocks():
     out3 = torch.zeros(4, 4, 64, dtype=torch.bfloat16, device="cuda:0")
     assert _raw_decode(wl3, p, out3) == pa.PA_OK
     assert pa.pa_device_status(clear=True) & pa.PA_DEV_BAD_ROW
+
+
+@pytest.mark.parametrize("seq_len", [64, 512, 4096, 16384])
+def test_executorch_h100_benchmark_shape(seq_len):
+    # ExecuTorch PR #18759's standalone kernel benchmark shape (B=1, H_q=16,
+    # H_kv=2, D=256, one decode token), here over a paged cache
+    wl = make_workload(seq_lens=[seq_len], query_lens=[1], num_q_heads=16, num_kv_heads=2,
+                       head_dim=256, block_size=16, seed=seq_len)
+    out = pa.decode(dev(wl))
+    check_full(wl, out, f"D=256 S={seq_len}")
+
+
+@pytest.mark.parametrize("block_size", [16, 1024])
+@pytest.mark.parametrize("parts", [0, 3, 80])
+def test_head_dim_256_mixed_rows_and_windows(block_size, parts):
+    wl = make_workload(seq_lens=[3000, 77, 1500, 300], query_lens=[1, 2, 4, 5], num_q_heads=8,
+                       num_kv_heads=2, head_dim=256, block_size=block_size,
+                       windows=[100, 0, 700, 16], seed=block_size + parts)
+    out = pa.decode(dev(wl), force_partitions=parts)
+    check_full(wl, out, f"D=256 BS={block_size} parts={parts}")
