@@ -175,6 +175,25 @@ int pa_visible_ranges(int32_t *lo, int32_t *hi, const int32_t *seqLens,
                       int batch, void *stream);
 
 /*
+ * pa_unreachable_blocks -- for every row, how many leading KV blocks no query
+ * token of this call or of any later call can see again.  With window w > 0
+ * a token at position p sees p-w+1 .. p, and later tokens sit at larger
+ * positions, so every block that ends at or before the row's earliest
+ * visible position, max(0, S-L+1-w), is dead: floor(that / kvBlockSize)
+ * blocks.  With w = 0 nothing is dead.  The cache still holds them; a
+ * caller's block allocator may free (and reuse) those blocks (gllm PR #116,
+ * "What changes": freeing blocks a window can no longer reach is left to a
+ * separate change).  Rows with queryLens[b] = 0 report 0.
+ *   count        device int32 [batch] (output)
+ *   seqLens, queryLens, windows (may be NULL)  device int32 [batch]
+ * Returns PA_ERR_ARG for null pointers, batch < 0 or window < 0, and
+ * PA_ERR_UNSUPPORTED for a block size outside [16, 1024] or not a power of two.
+ */
+int pa_unreachable_blocks(int32_t *count, const int32_t *seqLens, const int32_t *queryLens,
+                          int window, const int32_t *windows, int kvBlockSize, int batch,
+                          void *stream);
+
+/*
  * pa_decode_host -- end-to-end call with host buffers: copies q, blockTables,
  * seqLens, queryLens (and windows) from host memory into the caller's
  * workspace, runs pa_decode, copies dst back, and synchronises the stream.

@@ -56,6 +56,8 @@ def _load():
             lib.oracle_visible_range.restype = I
             lib.oracle_visible_ranges.argtypes = [P, P, P, P, P, I, I]
             lib.oracle_visible_ranges.restype = I
+            lib.oracle_unreachable_blocks.argtypes = [P, P, P, P, I, I, I]
+            lib.oracle_unreachable_blocks.restype = I
             lib.oracle_max_threads.argtypes = [I]
             lib.oracle_max_threads.restype = I
             common = [P, P, P, P, P, P, P, I, D, I, I, I, I, I, I, I]
@@ -180,3 +182,19 @@ def max_threads(nthreads: int = 0) -> int:
     """Threads the oracle's parallel loops use (OpenMP), after setting nthreads
     when it is positive."""
     return int(_load().oracle_max_threads(int(nthreads)))
+
+
+def unreachable_blocks(seq_lens, query_lens, block_size, window=0, windows=None):
+    """int32 [batch]: leading blocks of each row no current or later query
+    token can see."""
+    lib = _load()
+    seq_lens = _i32(seq_lens)
+    query_lens = _i32(query_lens)
+    windows = _i32(windows)
+    out = np.zeros(max(int(seq_lens.shape[0]), 1), dtype=np.int32)
+    rc = lib.oracle_unreachable_blocks(_ptr(out), _ptr(seq_lens), _ptr(query_lens),
+                                       _ptr(windows), int(window), int(block_size),
+                                       int(seq_lens.shape[0]))
+    if rc != 0:
+        raise ValueError("oracle rejected the lengths")
+    return out[:seq_lens.shape[0]]

@@ -114,6 +114,33 @@ int oracle_visible_ranges(int32_t *lo, int32_t *hi, const int32_t *seq_lens,
     return n;
 }
 
+/* Leading KV blocks of each row that no query token of this call, nor any
+ * later token of the row (later tokens sit at larger positions, so their
+ * windows start no earlier), can see: the blocks that end at or before the
+ * lowest visible position of the row's tokens.  Window 0 sees everything, so
+ * nothing is dead.  gllm PR #116 "feat(backend): sliding-window
+ * PagedAttention", "What changes": the cache keeps every position; freeing
+ * blocks a window can no longer reach is a separate step. */
+int oracle_unreachable_blocks(int32_t *count, const int32_t *seq_lens,
+                              const int32_t *query_lens, const int32_t *windows,
+                              int window, int bs, int batch)
+{
+    for (int b = 0; b < batch; ++b) {
+        int w = windows ? windows[b] : window;
+        count[b] = 0;
+        if (query_lens[b] <= 0 || w == 0) continue;
+        int lowest = seq_lens[b];
+        for (int i = 0; i < query_lens[b]; ++i) {
+            int lo, hi;
+            if (oracle_visible_range(seq_lens[b], query_lens[b], i, w, &lo, &hi))
+                return ORACLE_EINVAL;
+            if (lo < lowest) lowest = lo;
+        }
+        count[b] = lowest / bs;
+    }
+    return ORACLE_OK;
+}
+
 static int validate(const problem *pr)
 {
     if (pr->batch < 0 || pr->hq <= 0 || pr->hkv <= 0 || pr->d <= 0 ||

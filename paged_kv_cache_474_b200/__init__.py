@@ -90,6 +90,7 @@ SIGNATURES = {
     "pa_decode_host": (_I, [_P, _P, _P, _P, _P, _P, _P, _F, _I, _I, _PP, _P]),
     "pa_decode_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _F, _I, _I, _PP, _P]),
     "pa_host_workspace_size": (ctypes.c_size_t, [_PP, _I, _I, _P, _P]),
+    "pa_unreachable_blocks": (_I, [_P, _P, _P, _I, _P, _I, _I, _P]),
     "pa_extents_host": (_I, [_P, _P, _P, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I)]),
     "pa_device_status": (_I, [ctypes.POINTER(ctypes.c_uint), _I, _P]),
     "pa_last_error": (ctypes.c_char_p, []),
@@ -286,6 +287,23 @@ def decode(wl, *, out=None, workspace=None, hints=True, force_variant=PA_VARIANT
                      wl.v_cache.data_ptr(), wl.block_tables.data_ptr(),
                      wl.seq_lens.data_ptr(), wl.query_lens.data_ptr(), wl.scale,
                      wl.window, wl.block_size, p, _stream_handle(stream)))
+    return out
+
+
+def pa_unreachable_blocks(count, seqLens, queryLens, window, windows, kvBlockSize, batch,
+                          stream) -> int:
+    return _lib.pa_unreachable_blocks(count, seqLens, queryLens, int(window), windows,
+                                      int(kvBlockSize), int(batch), stream)
+
+
+def unreachable_blocks(seq_lens, query_lens, kv_block_size, window=0, windows=None, stream=None):
+    """int32 device tensor [batch]: leading KV blocks of each row that no query
+    token can see again (pa_unreachable_blocks)."""
+    import torch
+    out = torch.empty(seq_lens.numel(), dtype=torch.int32, device=seq_lens.device)
+    _check(pa_unreachable_blocks(out.data_ptr(), seq_lens.data_ptr(), query_lens.data_ptr(),
+                                 window, _ptr(windows), kv_block_size, seq_lens.numel(),
+                                 _stream_handle(stream)))
     return out
 
 

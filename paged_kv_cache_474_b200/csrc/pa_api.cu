@@ -495,6 +495,22 @@ int pa_visible_ranges(int32_t* lo, int32_t* hi, const int32_t* seqLens, const in
   return succeed();
 }
 
+int pa_unreachable_blocks(int32_t* count, const int32_t* seqLens, const int32_t* queryLens,
+                          int window, const int32_t* windows, int kvBlockSize, int batch,
+                          void* stream) {
+  if (!count || !seqLens || !queryLens) return fail(PA_ERR_ARG, "a required pointer is NULL");
+  if (batch < 0) return fail(PA_ERR_ARG, "batch %d is negative", batch);
+  if (window < 0) return fail(PA_ERR_ARG, "window %d is negative", window);
+  if (!is_pow2(kvBlockSize) || kvBlockSize < 16 || kvBlockSize > 1024)
+    return fail(PA_ERR_UNSUPPORTED, "kvBlockSize %d not supported (power of two in [16,1024])",
+                kvBlockSize);
+  if (batch == 0) return succeed();
+  cudaError_t e = pa::launch_unreachable(count, seqLens, queryLens, window, windows,
+                                         ilog2(kvBlockSize), batch, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "kernel launch: %s", cudaGetErrorString(e));
+  return succeed();
+}
+
 size_t pa_host_workspace_size(const pa_params* params, int kvBlockSize, int window,
                               const int32_t* seqLens_host, const int32_t* queryLens_host) {
   if (check_params(params, kvBlockSize) || !seqLens_host || !queryLens_host) return (size_t)-1;

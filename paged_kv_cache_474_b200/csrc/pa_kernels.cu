@@ -1052,6 +1052,21 @@ cudaError_t ensure_smem_attrs(const void* kern, size_t smem) {
   return cudaSuccess;
 }
 
+// Leading blocks of each row that its windowed query tokens (and later ones)
+// can no longer see: floor(union_lo / BS).
+__global__ void pa_unreachable_kernel(int32_t* count, const int32_t* seq_lens,
+                                      const int32_t* query_lens, int window, const int32_t* windows,
+                                      int block_shift, int batch) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= batch) return;
+  const int S = seq_lens[b], L = query_lens[b];
+  const int w = windows ? windows[b] : window;
+  int n = 0;
+  if (L > 0 && L <= S && w > 0) n = union_lo(S, L, w) >> block_shift;
+  if (L > S || L < 0 || w < 0) atomicOr(&g_pa_status, PA_DEV_BAD_ROW);
+  count[b] = n;
+}
+
 template <int D, int NCW, int NSTAGE>
 cudaError_t launch_fma_t(const DecodeArgs& a, dim3 grid, size_t smem, cudaStream_t stream) {
   auto kern = pa_partition_fma_kernel<D, NCW, NSTAGE>;
@@ -1207,6 +1222,14 @@ cudaError_t launch_ranges(int32_t* lo, int32_t* hi, const int32_t* seq_lens,
                           const int32_t* query_lens, int window, const int32_t* windows,
                           int batch, cudaStream_t stream) {
   pa_ranges_kernel<<<1, 1024, 0, stream>>>(lo, hi, seq_lens, query_lens, window, windows, batch);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unreachable(int32_t* count, const int32_t* seq_lens, const int32_t* query_lens,
+                               int window, const int32_t* windows, int block_shift, int batch,
+                               cudaStream_t stream) {
+  pa_unreachable_kernel<<<(batch + 255) / 256, 256, 0, stream>>>(count, seq_lens, query_lens, window,
+                                                                  windows, block_shift, batch);
   return cudaGetLastError();
 }
 

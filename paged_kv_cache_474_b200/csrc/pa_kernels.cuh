@@ -74,6 +74,11 @@ cudaError_t launch_ranges(int32_t* lo, int32_t* hi, const int32_t* seq_lens,
                           const int32_t* query_lens, int window, const int32_t* windows,
                           int batch, cudaStream_t stream);
 
+// Launches the dead-leading-block count per row.
+cudaError_t launch_unreachable(int32_t* count, const int32_t* seq_lens, const int32_t* query_lens,
+                               int window, const int32_t* windows, int block_shift, int batch,
+                               cudaStream_t stream);
+
 // Reads (and optionally clears) the device status word.
 cudaError_t read_status(unsigned int* status, bool clear, cudaStream_t stream);
 

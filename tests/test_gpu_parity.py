@@ -354,3 +354,19 @@ def test_head_dim_256_mixed_rows_and_windows(block_size, parts):
                        windows=[100, 0, 700, 16], seed=block_size + parts)
     out = pa.decode(dev(wl), force_partitions=parts)
     check_full(wl, out, f"D=256 BS={block_size} parts={parts}")
+
+
+def test_unreachable_blocks_match_oracle():
+    cases = [config_lengths(c) for c in (1, 2, 3, 4, 5)]
+    cases += [([300, 40], [5, 1], w, None) for w in (0, 1, 16, 100, 4096)]
+    rng = np.random.default_rng(8)
+    s = rng.integers(1, 70000, 500).tolist()
+    l = [int(min(x, y)) for x, y in zip(s, rng.integers(0, 6, 500).tolist())]
+    cases.append((s, l, 0, rng.choice([0, 1, 63, 64, 4096, 30000], 500).tolist()))
+    for bs in (16, 64, 1024):
+        for s, l, w, ws in cases:
+            S = torch.tensor(s, dtype=torch.int32, device="cuda:0")
+            L = torch.tensor(l, dtype=torch.int32, device="cuda:0")
+            W = None if ws is None else torch.tensor(ws, dtype=torch.int32, device="cuda:0")
+            got = pa.unreachable_blocks(S, L, bs, w, W).cpu().numpy()
+            assert np.array_equal(got, oracle.unreachable_blocks(s, l, bs, w, ws))

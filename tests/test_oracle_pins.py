@@ -340,3 +340,37 @@ def test_empty_query_rows_produce_no_outputs():
     assert got.shape == (2, 2, 8)
     ref = sdpa_reference(w, lambda b: 0)
     assert np.max(np.abs(got - ref)) <= 1e-12
+
+
+def test_unreachable_blocks_match_brute_force():
+    # A block is dead when no position in it is visible to any query token of
+    # the row now or later (later tokens only move the window right): brute
+    # force over every position of every leading block.
+    rng = np.random.default_rng(4)
+    for _ in range(300):
+        bs = int(rng.choice([16, 32, 1024]))
+        S = int(rng.integers(1, 6000))
+        L = int(rng.integers(0, min(S, 6) + 1))
+        w = int(rng.choice([0, 1, 5, 16, 100, 4096, int(rng.integers(1, 7000))]))
+        got = int(oracle.unreachable_blocks([S], [L], bs, w)[0])
+        want = 0
+        if L > 0 and w > 0:
+            for j in range((S + bs - 1) // bs):
+                seen = False
+                for p_ in range(S - L, S + 3):   # current tokens and a few later ones
+                    lo = max(0, p_ + 1 - w)
+                    if any(lo <= t <= p_ for t in range(j * bs, (j + 1) * bs)):
+                        seen = True
+                        break
+                if seen:
+                    break
+                want += 1
+        assert got == want, (S, L, w, bs)
+
+
+def test_unreachable_blocks_on_the_gllm_batch():
+    # 5-token chunk over 300 and a decode row over 40, 16-token blocks
+    assert oracle.unreachable_blocks([300, 40], [5, 1], 16, 16).tolist() == [17, 1]
+    assert oracle.unreachable_blocks([300, 40], [5, 1], 16, 100).tolist() == [12, 0]
+    assert oracle.unreachable_blocks([300, 40], [5, 1], 16, 0).tolist() == [0, 0]
+    assert oracle.unreachable_blocks([300, 40], [0, 1], 16, windows=[16, 4096]).tolist() == [0, 0]
