@@ -60,7 +60,9 @@ def _load():
             lib.oracle_unreachable_blocks.restype = I
             lib.oracle_max_threads.argtypes = [I]
             lib.oracle_max_threads.restype = I
-            common = [P, P, P, P, P, P, P, I, D, I, I, I, I, I, I, I]
+            common = [P, P, P, P, P, P, P, I, D, I, I, I, I, I, I, I, I, D, D]
+            lib.oracle_e4m3_decode.argtypes = [P, P, I]
+            lib.oracle_e4m3_decode.restype = None
             lib.oracle_pa_decode.argtypes = [P] + common + [I, I]
             lib.oracle_pa_decode.restype = I
             lib.oracle_pa_decode_select.argtypes = [P, P, I] + common + [I]
@@ -90,17 +92,28 @@ class Problem:
     """One paged-attention decode problem, as host arrays.
 
     q:            uint16 [sum(query_lens), H_q, D]   (bf16 bits)
-    k_cache/v_cache: uint16 [num_blocks, H_kv, block_size, D]
+    k_cache/v_cache: uint16 [num_blocks, H_kv, block_size, D] (bf16 bits), or
+                  uint8 of the same shape (FP8 e4m3 codes; the value of a code
+                  is its e4m3 number times k_scale / v_scale)
     block_tables: int32 [batch, max_blocks_per_seq]
     seq_lens, query_lens: int32 [batch]
     windows:      int32 [batch] or None (then the scalar ``window`` applies)
     """
 
     def __init__(self, q, k_cache, v_cache, block_tables, seq_lens, query_lens,
-                 scale, window=0, windows=None):
+                 scale, window=0, windows=None, k_scale=1.0, v_scale=1.0):
         self.q = _u16(q)
-        self.k_cache = _u16(k_cache)
-        self.v_cache = _u16(v_cache)
+        k_cache = np.ascontiguousarray(k_cache)
+        v_cache = np.ascontiguousarray(v_cache)
+        self.kv_fp8 = int(k_cache.dtype == np.uint8)
+        if self.kv_fp8:
+            if v_cache.dtype != np.uint8:
+                raise TypeError("k_cache and v_cache must both be FP8 codes")
+            self.k_cache, self.v_cache = k_cache, v_cache
+        else:
+            self.k_cache, self.v_cache = _u16(k_cache), _u16(v_cache)
+        self.k_scale = float(k_scale)
+        self.v_scale = float(v_scale)
         self.block_tables = _i32(block_tables)
         self.seq_lens = _i32(seq_lens)
         self.query_lens = _i32(query_lens)
@@ -120,7 +133,7 @@ class Problem:
                 _ptr(self.block_tables), _ptr(self.seq_lens),
                 _ptr(self.query_lens), _ptr(self.windows), self.window,
                 self.scale, self.batch, self.hq, self.hkv, self.d, self.bs,
-                self.num_blocks, self.mbps]
+                self.num_blocks, self.mbps, self.kv_fp8, self.k_scale, self.v_scale]
 
     @property
     def num_tokens(self) -> int:
@@ -198,3 +211,12 @@ def unreachable_blocks(seq_lens, query_lens, block_size, window=0, windows=None)
     if rc != 0:
         raise ValueError("oracle rejected the lengths")
     return out[:seq_lens.shape[0]]
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """float64 values of FP8 e4m3 codes (uint8), decoded by the oracle."""
+    lib = _load()
+    codes = np.ascontiguousarray(np.asarray(codes, dtype=np.uint8))
+    out = np.zeros(codes.shape, dtype=np.float64)
+    lib.oracle_e4m3_decode(_ptr(out), _ptr(codes), int(codes.size))
+    return out

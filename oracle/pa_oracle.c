@@ -61,13 +61,42 @@ static double bf16_bits_to_double(uint16_t h)
     return (double)f;
 }
 
+/* FP8 e4m3 bit pattern -> double: sign, 4-bit exponent (bias 7), 3-bit
+ * mantissa; exponent 0 is subnormal (m/8 * 2^-6); the two codes with every
+ * exponent and mantissa bit set are NaN; there is no infinity. */
+static double e4m3_bits_to_double(uint8_t x)
+{
+    int sign = x >> 7, e = (x >> 3) & 15, m = x & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m / 8.0, -6);
+    else v = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
 typedef struct {
-    const uint16_t *q, *kc, *vc;
+    const uint16_t *q;
+    const void *kc, *vc;   /* bf16 (uint16) or, with kv_fp8, e4m3 (uint8) elements */
     const int32_t *block_tables, *seq_lens, *query_lens, *windows;
     int window;
     double scale;
     int batch, hq, hkv, d, bs, num_blocks, mbps;
+    int kv_fp8;            /* caches hold e4m3 codes; value = code * k_scale (v_scale) */
+    double k_scale, v_scale;
 } problem;
+
+/* Element idx of a cache as a double (dequantised for FP8 caches). */
+static double kv_value(const problem *pr, const void *cache, size_t idx, double s)
+{
+    if (pr->kv_fp8) return s * e4m3_bits_to_double(((const uint8_t *)cache)[idx]);
+    return bf16_bits_to_double(((const uint16_t *)cache)[idx]);
+}
+
+/* Exported for the tests: decodes n e4m3 codes. */
+void oracle_e4m3_decode(double *out, const uint8_t *codes, int n)
+{
+    for (int i = 0; i < n; ++i) out[i] = e4m3_bits_to_double(codes[i]);
+}
 
 static int row_window(const problem *pr, int b)
 {
@@ -175,10 +204,10 @@ static size_t cache_index(const problem *pr, int b, int g, int t)
  * scale * sum_d q[d] * k_t[d]. */
 static double score(const problem *pr, const uint16_t *qrow, int b, int g, int t)
 {
-    const uint16_t *k = pr->kc + cache_index(pr, b, g, t);
+    const size_t k = cache_index(pr, b, g, t);
     double acc = 0.0;
     for (int x = 0; x < pr->d; ++x)
-        acc += bf16_bits_to_double(qrow[x]) * bf16_bits_to_double(k[x]);
+        acc += bf16_bits_to_double(qrow[x]) * kv_value(pr, pr->kc, k + x, pr->k_scale);
     return pr->scale * acc;
 }
 
@@ -219,8 +248,8 @@ static double attend_range(const problem *pr, int b, int i, int h, int t0,
     for (int t = t0; t < t1; ++t) {
         double a = exp(s[t - t0] - m) / z;
         if (w) w[t - t0] = a;
-        const uint16_t *v = pr->vc + cache_index(pr, b, g, t);
-        for (int x = 0; x < pr->d; ++x) out[x] += a * bf16_bits_to_double(v[x]);
+        const size_t v = cache_index(pr, b, g, t);
+        for (int x = 0; x < pr->d; ++x) out[x] += a * kv_value(pr, pr->vc, v + x, pr->v_scale);
     }
     free(s);
     return m + log(z);
@@ -305,16 +334,17 @@ int oracle_max_threads(int nthreads)
 /* Every output: out is [sum(queryLens)][H_q][head_dim] doubles.
  * parts == 0: direct two-pass softmax; parts > 0: split-K with that many
  * partitions per row, merged by log-sum-exp. */
-int oracle_pa_decode(double *out, const uint16_t *q, const uint16_t *kc,
-                     const uint16_t *vc, const int32_t *block_tables,
+int oracle_pa_decode(double *out, const uint16_t *q, const void *kc,
+                     const void *vc, const int32_t *block_tables,
                      const int32_t *seq_lens, const int32_t *query_lens,
                      const int32_t *windows, int window, double scale,
                      int batch, int hq, int hkv, int d, int bs, int num_blocks,
-                     int max_blocks_per_seq, int parts, int nthreads)
+                     int max_blocks_per_seq, int kv_fp8, double k_scale, double v_scale,
+                     int parts, int nthreads)
 {
     problem pr = {q, kc, vc, block_tables, seq_lens, query_lens, windows,
                   window, scale, batch, hq, hkv, d, bs, num_blocks,
-                  max_blocks_per_seq};
+                  max_blocks_per_seq, kv_fp8, k_scale, v_scale};
     if (validate(&pr) || parts < 0) return ORACLE_EINVAL;
     /* list every (b, i, h) with its output slot */
     size_t ntok = 0;
@@ -340,16 +370,17 @@ int oracle_pa_decode(double *out, const uint16_t *q, const uint16_t *kc,
 
 /* A chosen subset of outputs: sel is [nsel][3] (b, i, h); out is [nsel][d]. */
 int oracle_pa_decode_select(double *out, const int32_t *sel, int nsel,
-                            const uint16_t *q, const uint16_t *kc,
-                            const uint16_t *vc, const int32_t *block_tables,
+                            const uint16_t *q, const void *kc,
+                            const void *vc, const int32_t *block_tables,
                             const int32_t *seq_lens, const int32_t *query_lens,
                             const int32_t *windows, int window, double scale,
                             int batch, int hq, int hkv, int d, int bs,
-                            int num_blocks, int max_blocks_per_seq, int nthreads)
+                            int num_blocks, int max_blocks_per_seq, int kv_fp8,
+                            double k_scale, double v_scale, int nthreads)
 {
     problem pr = {q, kc, vc, block_tables, seq_lens, query_lens, windows,
                   window, scale, batch, hq, hkv, d, bs, num_blocks,
-                  max_blocks_per_seq};
+                  max_blocks_per_seq, kv_fp8, k_scale, v_scale};
     if (validate(&pr)) return ORACLE_EINVAL;
     for (int j = 0; j < nsel; ++j) {
         int b = sel[3 * j], i = sel[3 * j + 1], h = sel[3 * j + 2];
@@ -368,15 +399,16 @@ int oracle_pa_decode_select(double *out, const int32_t *sel, int nsel,
 /* Softmax weights of one query (b, i, h) over every cached position of its
  * row: w is [seq_lens[b]] doubles, zero outside the visible range. */
 int oracle_softmax_weights(double *w, int b, int i, int h, const uint16_t *q,
-                           const uint16_t *kc, const uint16_t *vc,
+                           const void *kc, const void *vc,
                            const int32_t *block_tables, const int32_t *seq_lens,
                            const int32_t *query_lens, const int32_t *windows,
                            int window, double scale, int batch, int hq, int hkv,
-                           int d, int bs, int num_blocks, int max_blocks_per_seq)
+                           int d, int bs, int num_blocks, int max_blocks_per_seq,
+                           int kv_fp8, double k_scale, double v_scale)
 {
     problem pr = {q, kc, vc, block_tables, seq_lens, query_lens, windows,
                   window, scale, batch, hq, hkv, d, bs, num_blocks,
-                  max_blocks_per_seq};
+                  max_blocks_per_seq, kv_fp8, k_scale, v_scale};
     if (validate(&pr)) return ORACLE_EINVAL;
     if (b < 0 || b >= batch || i < 0 || i >= query_lens[b] || h < 0 || h >= hq)
         return ORACLE_EINVAL;

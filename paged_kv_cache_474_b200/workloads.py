@@ -24,7 +24,9 @@ sum(ceil(S_b/BS)) blocks plus one spare; the pool is randomly permuted and
 handed out to the rows in row order; unused block-table slots hold 0.
 Values are drawn as float32 (uniform(-1,1) for the tiny workload, standard
 normal otherwise) on the requested device and rounded to bf16 (round to
-nearest even); both sides then read the same bf16 bytes.
+nearest even); both sides then read the same bf16 bytes.  FP8 caches
+(kv_dtype="fp8_e4m3") quantise those bf16 values per tensor: scale =
+max|x| / 448, codes = round-to-nearest e4m3 of x / scale.
 """
 from __future__ import annotations
 
@@ -58,6 +60,14 @@ class Workload:
     window: int
     scale: float
     name: str = ""
+    # FP8 caches: k_cache / v_cache hold e4m3 codes (torch.uint8); a code's
+    # value is its e4m3 number times k_scale / v_scale.  1.0 for bf16 caches.
+    k_scale: float = 1.0
+    v_scale: float = 1.0
+
+    @property
+    def kv_fp8(self) -> bool:
+        return self.k_cache.dtype == torch.uint8
 
     @property
     def batch(self) -> int:
@@ -108,8 +118,12 @@ class Workload:
 
 
 def bf16_bits(t: torch.Tensor) -> np.ndarray:
-    """Host numpy uint16 view of a bf16 tensor's bit patterns."""
-    return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+    """Host numpy view of a cache or q tensor's bit patterns: uint16 for bf16,
+    uint8 for FP8 codes (already uint8)."""
+    t = t.detach().contiguous().cpu()
+    if t.dtype == torch.uint8:
+        return t.numpy()
+    return t.view(torch.int16).numpy().view(np.uint16)
 
 
 def _gen(seed: int, device) -> torch.Generator:
@@ -135,13 +149,24 @@ def _values(shape, dist: str, g: torch.Generator, device):
     return out
 
 
+def to_e4m3(x: torch.Tensor):
+    """Per-tensor FP8 e4m3 codes of x (uint8) and their scale: the scale
+    maps the largest |x| to 448, the largest finite e4m3 number; torch's
+    float8_e4m3fn cast rounds to nearest."""
+    amax = float(x.abs().max()) if x.numel() else 1.0
+    s = (amax / 448.0) if amax > 0 else 1.0
+    codes = (x.float() / s).to(torch.float8_e4m3fn).view(torch.uint8)
+    return codes, s
+
+
 def make_workload(*, seq_lens: Sequence[int], query_lens: Sequence[int],
                   num_q_heads: int, num_kv_heads: int, head_dim: int,
                   block_size: int, window: int = 0,
                   windows: Optional[Sequence[int]] = None,
                   scale: Optional[float] = None, dist: str = "normal",
                   seed: int = 0, device="cpu", spare_blocks: int = 1,
-                  extra_table_cols: int = 0, name: str = "") -> Workload:
+                  extra_table_cols: int = 0, name: str = "",
+                  kv_dtype: str = "bf16") -> Workload:
     """Build a workload with explicit lengths.  Blocks are a random permutation
     of a pool of sum(ceil(S_b/BS)) + spare_blocks blocks handed out in row
     order; unused block-table slots (and ``extra_table_cols`` padding columns)
@@ -170,11 +195,18 @@ def make_workload(*, seq_lens: Sequence[int], query_lens: Sequence[int],
     if scale is None:
         scale = 1.0 / math.sqrt(head_dim)
     win_t = None if windows is None else torch.tensor(list(windows), dtype=torch.int32)
+    ks = vs = 1.0
+    if kv_dtype == "fp8_e4m3":
+        k, ks = to_e4m3(k)
+        v, vs = to_e4m3(v)
+    elif kv_dtype != "bf16":
+        raise ValueError(f"unknown kv_dtype {kv_dtype}")
     return Workload(q=q, k_cache=k, v_cache=v, block_tables=tables.to(device),
                     seq_lens=torch.tensor(seq_lens, dtype=torch.int32).to(device),
                     query_lens=torch.tensor(query_lens, dtype=torch.int32).to(device),
                     windows=None if win_t is None else win_t.to(device),
-                    window=int(window), scale=float(scale), name=name)
+                    window=int(window), scale=float(scale), name=name,
+                    k_scale=float(ks), v_scale=float(vs))
 
 
 def config_lengths(cfg: int):
@@ -208,12 +240,14 @@ _SHAPES = {
 }
 
 
-def config_workload(cfg: int, device="cpu", window: Optional[int] = None) -> Workload:
+def config_workload(cfg: int, device="cpu", window: Optional[int] = None,
+                    kv_dtype: str = "bf16") -> Workload:
     """One of the five named workloads.  ``window`` overrides the scalar window
-    (the tiny workload is run at window 0 and window 8)."""
+    (the tiny workload is run at window 0 and window 8); kv_dtype="fp8_e4m3"
+    quantises its caches to per-tensor-scaled FP8."""
     s, l, w, ws = config_lengths(cfg)
     if window is not None:
         w = int(window)
     return make_workload(seq_lens=s, query_lens=l, window=w, windows=ws,
                          seed=4740 + cfg, device=device, name=CONFIG_NAMES[cfg],
-                         **_SHAPES[cfg])
+                         kv_dtype=kv_dtype, **_SHAPES[cfg])

@@ -12,7 +12,12 @@ Each test fixes the oracle to a fact from the pages or from mathematics:
     "scattered out-of-order blocks"), any split-K partition count gives the
     same result (ExecuTorch PR #18759, split-K merge), softmax weights sum to
     one and vanish outside the visible range;
-  - the hand-derived visible ranges in tests/golden/visible_ranges.txt.
+  - the hand-derived visible ranges in tests/golden/visible_ranges.txt;
+  - FP8 e4m3 caches: every one of the 256 codes decodes to the value torch's
+    float8_e4m3fn conversion gives, a handful of codes to their closed forms
+    (OCP 8-bit floating point formats: bias 7, no infinities, 448 largest),
+    and attention over FP8 codes equals float64 SDPA over the dequantised
+    caches, with k_scale acting on the logits and v_scale on the output.
 A plausible slip in the oracle (a dropped scale, an off-by-one window edge, a
 wrong GQA head map, a swapped K/V, a bad block lookup) fails at least one.
 """
@@ -35,7 +40,16 @@ def problem_of(w, window=None, windows="keep"):
         bf16_bits(w.q), bf16_bits(w.k_cache), bf16_bits(w.v_cache),
         w.block_tables.numpy(), w.seq_lens.numpy(), w.query_lens.numpy(),
         w.scale, w.window if window is None else window,
-        None if ws is None else np.asarray(ws, dtype=np.int32))
+        None if ws is None else np.asarray(ws, dtype=np.int32),
+        k_scale=w.k_scale, v_scale=w.v_scale)
+
+
+def cache_values(c, s):
+    """float64 values of a cache: bf16 as is, FP8 codes decoded by torch's own
+    float8_e4m3fn conversion and multiplied by their per-tensor scale."""
+    if c.dtype == torch.uint8:
+        return c.view(torch.float8_e4m3fn).double() * s
+    return c.double()
 
 
 def dense_kv(w, b):
@@ -43,8 +57,8 @@ def dense_kv(w, b):
     table (written here independently of the oracle)."""
     S = int(w.seq_lens[b])
     bs = w.block_size
-    kc = w.k_cache.double()
-    vc = w.v_cache.double()
+    kc = cache_values(w.k_cache, w.k_scale)
+    vc = cache_values(w.v_cache, w.v_scale)
     ks, vs = [], []
     for t in range(S):
         phys = int(w.block_tables[b, t // bs])
@@ -374,3 +388,69 @@ def test_unreachable_blocks_on_the_gllm_batch():
     assert oracle.unreachable_blocks([300, 40], [5, 1], 16, 100).tolist() == [12, 0]
     assert oracle.unreachable_blocks([300, 40], [5, 1], 16, 0).tolist() == [0, 0]
     assert oracle.unreachable_blocks([300, 40], [0, 1], 16, windows=[16, 4096]).tolist() == [0, 0]
+
+
+def test_e4m3_decode_matches_torch_for_every_code():
+    codes = np.arange(256, dtype=np.uint8)
+    got = oracle.e4m3_decode(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    nan = np.isnan(ref)
+    assert list(np.flatnonzero(nan)) == [0x7F, 0xFF]
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+
+
+@pytest.mark.parametrize("code,value", [
+    (0x00, 0.0), (0x38, 1.0), (0xB8, -1.0), (0x7E, 448.0), (0xFE, -448.0),
+    (0x08, 2.0 ** -6), (0x01, 2.0 ** -9), (0x07, 7 * 2.0 ** -9),
+    (0x3C, 1.5), (0x41, 2.25), (0x57, 15.0)])
+def test_e4m3_closed_forms(code, value):
+    # sign | 4 exponent bits (bias 7) | 3 mantissa bits; exponent 0 is subnormal
+    got = oracle.e4m3_decode(np.array([code], dtype=np.uint8))[0]
+    assert got == value
+    if code == 0x00:
+        assert not math.copysign(1.0, oracle.e4m3_decode(np.array([0x80], np.uint8))[0]) > 0
+
+
+def fp8_mixed(window=0, windows=None, seed=13):
+    return make_workload(seq_lens=[9, 23, 5, 31], query_lens=[1, 3, 5, 2],
+                         num_q_heads=6, num_kv_heads=2, head_dim=16,
+                         block_size=4, window=window, windows=windows,
+                         dist="normal", seed=seed, scale=0.3, kv_dtype="fp8_e4m3")
+
+
+@pytest.mark.parametrize("window,windows", [(0, None), (5, None), (4, [3, 0, 4, 7])])
+def test_fp8_caches_match_sdpa_on_dequantised_values(window, windows):
+    w = fp8_mixed(window, windows)
+    assert w.kv_fp8 and w.k_scale != w.v_scale
+    got = oracle.decode(problem_of(w))
+    wof = (lambda b: windows[b]) if windows is not None else (lambda b: window)
+    ref = sdpa_reference(w, wof)
+    assert np.max(np.abs(got - ref)) <= 1e-12
+
+
+def test_fp8_scales_act_on_logits_and_output():
+    w = fp8_mixed()
+    base = problem_of(w)
+    o = oracle.decode(base)
+    args = (base.q, base.k_cache, base.v_cache, base.block_tables, base.seq_lens,
+            base.query_lens)
+    # v_scale is a factor on every output (a power of two keeps it exact)
+    o2 = oracle.decode(oracle.Problem(*args, w.scale, k_scale=w.k_scale,
+                                      v_scale=2 * w.v_scale))
+    assert np.array_equal(o2, 2 * o)
+    # k_scale enters only through the logits: k_scale*c is the same as scale*c
+    o3 = oracle.decode(oracle.Problem(*args, w.scale * 1.7, k_scale=w.k_scale,
+                                      v_scale=w.v_scale))
+    o4 = oracle.decode(oracle.Problem(*args, w.scale, k_scale=w.k_scale * 1.7,
+                                      v_scale=w.v_scale))
+    assert np.max(np.abs(o3 - o4)) <= 1e-13
+    assert np.max(np.abs(o3 - o)) > 1e-3
+
+
+def test_fp8_split_k_invariance():
+    w = fp8_mixed(window=7)
+    pr = problem_of(w)
+    o = oracle.decode(pr)
+    for parts in (1, 2, 5):
+        assert np.max(np.abs(oracle.decode(pr, parts=parts) - o)) <= 1e-13
