@@ -24,7 +24,17 @@
  * directly and needs no temporaries (aiter PR #2914 "Pa gluon swa mtp opt",
  * the one_shot path).
  *
- * Layouts (all row-major, element type bf16 unless noted):
+ * FP8 operands (aiter PR #2914 "Pa gluon swa mtp opt", the review of
+ * pa_decode_gluon's scale arguments: an FP8 query comes with query_scale, FP8
+ * KV caches with key_scale and value_scale, and a missing scale must be
+ * rejected rather than silently ignored).  With pa_params.kv_dtype = PA_DTYPE_FP8_E4M3 the caches hold FP8
+ * e4m3 codes (OCP 8-bit format: 1 sign, 4 exponent bits with bias 7, 3
+ * mantissa bits, no infinities) and k_t, v_t above are the codes' values
+ * times the per-tensor k_scale, v_scale; with q_dtype = PA_DTYPE_FP8_E4M3, q
+ * holds codes and q is their value times q_scale.  dst stays bf16.
+ *
+ * Layouts (all row-major, element type bf16 unless noted; FP8 codes are one
+ * byte each, in the same shapes):
  *   q, dst        [sum(queryLens)][H_q][head_dim], rows packed in batch order
  *   kCache,vCache [num_blocks][H_kv][kvBlockSize][head_dim]
  *   blockTables   int32 [batch][max_blocks_per_seq]; only the first
@@ -65,6 +75,10 @@ extern "C" {
 #define PA_DEV_BAD_BLOCK 4u   /* a block-table entry outside [0, num_blocks) */
 #define PA_DEV_HINT 8u        /* a row longer than max_span_hint / max_query_len_hint */
 
+/* Operand types (pa_params.q_dtype, pa_params.kv_dtype). */
+#define PA_DTYPE_BF16 0
+#define PA_DTYPE_FP8_E4M3 1   /* per-tensor scaled FP8 e4m3 codes (tensor-core variant) */
+
 /* Kernel variants (pa_params.force_variant, pa_plan_info.variant). */
 #define PA_VARIANT_AUTO 0
 #define PA_VARIANT_FMA 1      /* CUDA-core FMA scores and PV (group x queryLen <= 4 rows) */
@@ -93,6 +107,18 @@ typedef struct pa_params {
      * pa_decode records on the stream immediately before and after the
      * partition kernel (the reduce, if any, runs after the second). */
     void *const *profile_events;
+    /* Operand types: PA_DTYPE_BF16 (0, the default) or PA_DTYPE_FP8_E4M3.
+     * A scale is read only for an FP8 operand and must then be finite and
+     * > 0: the zero of a zero-initialised struct means "not given" and is
+     * rejected.  FP8 runs on the tensor-core variant only (force_variant FMA
+     * with an FP8 operand is PA_ERR_UNSUPPORTED); with FP8 caches its MMAs
+     * take f16 operands, so a bf16 q must lie within f16's range (|q| <
+     * 65504). */
+    int q_dtype;
+    int kv_dtype;
+    float q_scale;
+    float k_scale;
+    float v_scale;
 } pa_params;
 
 /* What the dispatcher chose for a call (pa_plan). */
@@ -117,8 +143,8 @@ typedef struct pa_plan_info {
  *
  *   dst          device bf16 [sum(queryLens)][H_q][head_dim], written for rows
  *                with queryLens[b] > 0; other memory is untouched
- *   q            device bf16 [sum(queryLens)][H_q][head_dim]
- *   kCache,vCache device bf16 [num_blocks][H_kv][kvBlockSize][head_dim]
+ *   q            device bf16 (or FP8 codes, q_dtype) [sum(queryLens)][H_q][head_dim]
+ *   kCache,vCache device bf16 (or FP8 codes, kv_dtype) [num_blocks][H_kv][kvBlockSize][head_dim]
  *   blockTables  device int32 [batch][max_blocks_per_seq]
  *   seqLens      device int32 [batch], cached tokens per row (includes the new ones)
  *   queryLens    device int32 [batch], new query tokens per row (0 skips the row)
@@ -130,7 +156,8 @@ typedef struct pa_plan_info {
  *   stream       cudaStream_t
  *
  * All device pointers must be 16-byte aligned.  Returns PA_ERR_ARG for null
- * pointers, H_q % H_kv != 0, negative window or hints, misalignment;
+ * pointers, H_q % H_kv != 0, negative window or hints, misalignment, an
+ * unknown dtype, a missing or non-finite scale of an FP8 operand;
  * PA_ERR_UNSUPPORTED for head_dim not in {64,128,256} or a block size outside
  * the set above; PA_ERR_WORKSPACE when split-K partials are needed and the
  * workspace is too small; PA_ERR_CUDA when a launch fails.
@@ -199,7 +226,8 @@ int pa_unreachable_blocks(int32_t *count, const int32_t *seqLens, const int32_t 
  * workspace, runs pa_decode, copies dst back, and synchronises the stream.
  * The KV caches stay on the device (they are resident state).  Host buffers
  * should be pinned for asynchronous copies.
- *   dst_host, q_host  host bf16 [sum(queryLens)][H_q][head_dim]
+ *   dst_host          host bf16 [sum(queryLens)][H_q][head_dim]
+ *   q_host            host bf16 or FP8 codes (q_dtype), same shape
  *   blockTables_host, seqLens_host, queryLens_host  host int32
  *   params->windows   host int32 [batch] or NULL (host memory in this call)
  *   params->workspace device, >= pa_host_workspace_size() bytes

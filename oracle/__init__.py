@@ -7,7 +7,8 @@ back here.
 
 The arithmetic lives in ``pa_oracle.c`` (plain C, float64, optional OpenMP);
 this module builds it with gcc and marshals numpy arrays through ctypes.
-Inputs are bf16 bit patterns (``numpy.uint16``), exactly as the GPU sees them.
+Inputs are bf16 bit patterns (``numpy.uint16``) or FP8 e4m3 codes
+(``numpy.uint8``, with per-tensor scales), exactly as the GPU sees them.
 
 Sources: gllm PR #116 "feat(backend): sliding-window PagedAttention"
 (sections "What changes" and "Verification") for the call, the window rule
@@ -60,7 +61,7 @@ def _load():
             lib.oracle_unreachable_blocks.restype = I
             lib.oracle_max_threads.argtypes = [I]
             lib.oracle_max_threads.restype = I
-            common = [P, P, P, P, P, P, P, I, D, I, I, I, I, I, I, I, I, D, D]
+            common = [P, P, P, P, P, P, P, I, D, I, I, I, I, I, I, I, I, D, D, I, D]
             lib.oracle_e4m3_decode.argtypes = [P, P, I]
             lib.oracle_e4m3_decode.restype = None
             lib.oracle_pa_decode.argtypes = [P] + common + [I, I]
@@ -91,7 +92,8 @@ def _i32(a):
 class Problem:
     """One paged-attention decode problem, as host arrays.
 
-    q:            uint16 [sum(query_lens), H_q, D]   (bf16 bits)
+    q:            uint16 [sum(query_lens), H_q, D]   (bf16 bits), or uint8
+                  FP8 e4m3 codes (value = e4m3 number times q_scale)
     k_cache/v_cache: uint16 [num_blocks, H_kv, block_size, D] (bf16 bits), or
                   uint8 of the same shape (FP8 e4m3 codes; the value of a code
                   is its e4m3 number times k_scale / v_scale)
@@ -101,8 +103,12 @@ class Problem:
     """
 
     def __init__(self, q, k_cache, v_cache, block_tables, seq_lens, query_lens,
-                 scale, window=0, windows=None, k_scale=1.0, v_scale=1.0):
-        self.q = _u16(q)
+                 scale, window=0, windows=None, k_scale=1.0, v_scale=1.0,
+                 q_scale=1.0):
+        q = np.ascontiguousarray(q)
+        self.q_fp8 = int(q.dtype == np.uint8)
+        self.q = q if self.q_fp8 else _u16(q)
+        self.q_scale = float(q_scale)
         k_cache = np.ascontiguousarray(k_cache)
         v_cache = np.ascontiguousarray(v_cache)
         self.kv_fp8 = int(k_cache.dtype == np.uint8)
@@ -133,7 +139,8 @@ class Problem:
                 _ptr(self.block_tables), _ptr(self.seq_lens),
                 _ptr(self.query_lens), _ptr(self.windows), self.window,
                 self.scale, self.batch, self.hq, self.hkv, self.d, self.bs,
-                self.num_blocks, self.mbps, self.kv_fp8, self.k_scale, self.v_scale]
+                self.num_blocks, self.mbps, self.kv_fp8, self.k_scale, self.v_scale,
+                self.q_fp8, self.q_scale]
 
     @property
     def num_tokens(self) -> int:

@@ -36,6 +36,11 @@
  *  - scale is used exactly as passed.
  *  - windows[b], when given, overrides the scalar window for row b.
  *
+ * FP8 operands (aiter PR #2914 "Pa gluon swa mtp opt", review of
+ * pa_decode_gluon's query_scale / key_scale / value_scale): an FP8 query or
+ * FP8 caches hold e4m3 codes, and an element's value is its code's number
+ * times the tensor's scale.
+ *
  * Arithmetic: inputs are bf16 bit patterns, widened exactly to double; every
  * sum, exponential and division is done in double, in the two-pass form of
  * the definition (exact maximum first, then the normalised sum).
@@ -75,7 +80,7 @@ static double e4m3_bits_to_double(uint8_t x)
 }
 
 typedef struct {
-    const uint16_t *q;
+    const void *q;         /* bf16 (uint16) or, with q_fp8, e4m3 (uint8) elements */
     const void *kc, *vc;   /* bf16 (uint16) or, with kv_fp8, e4m3 (uint8) elements */
     const int32_t *block_tables, *seq_lens, *query_lens, *windows;
     int window;
@@ -83,6 +88,8 @@ typedef struct {
     int batch, hq, hkv, d, bs, num_blocks, mbps;
     int kv_fp8;            /* caches hold e4m3 codes; value = code * k_scale (v_scale) */
     double k_scale, v_scale;
+    int q_fp8;             /* q holds e4m3 codes; value = code * q_scale */
+    double q_scale;
 } problem;
 
 /* Element idx of a cache as a double (dequantised for FP8 caches). */
@@ -90,6 +97,13 @@ static double kv_value(const problem *pr, const void *cache, size_t idx, double 
 {
     if (pr->kv_fp8) return s * e4m3_bits_to_double(((const uint8_t *)cache)[idx]);
     return bf16_bits_to_double(((const uint16_t *)cache)[idx]);
+}
+
+/* Element idx of q as a double (dequantised for an FP8 query). */
+static double q_value(const problem *pr, size_t idx)
+{
+    if (pr->q_fp8) return pr->q_scale * e4m3_bits_to_double(((const uint8_t *)pr->q)[idx]);
+    return bf16_bits_to_double(((const uint16_t *)pr->q)[idx]);
 }
 
 /* Exported for the tests: decodes n e4m3 codes. */
@@ -202,12 +216,12 @@ static size_t cache_index(const problem *pr, int b, int g, int t)
 
 /* Score of query (row b, token i, head h) against cached token t:
  * scale * sum_d q[d] * k_t[d]. */
-static double score(const problem *pr, const uint16_t *qrow, int b, int g, int t)
+static double score(const problem *pr, size_t qrow, int b, int g, int t)
 {
     const size_t k = cache_index(pr, b, g, t);
     double acc = 0.0;
     for (int x = 0; x < pr->d; ++x)
-        acc += bf16_bits_to_double(qrow[x]) * kv_value(pr, pr->kc, k + x, pr->k_scale);
+        acc += q_value(pr, qrow + x) * kv_value(pr, pr->kc, k + x, pr->k_scale);
     return pr->scale * acc;
 }
 
@@ -228,7 +242,7 @@ static double attend_range(const problem *pr, int b, int i, int h, int t0,
                            int t1, double *out, double *w)
 {
     int g = h / (pr->hq / pr->hkv);
-    const uint16_t *qrow = pr->q + qrow_offset(pr, b, i, h);
+    const size_t qrow = qrow_offset(pr, b, i, h);
     for (int x = 0; x < pr->d; ++x) out[x] = 0.0;
     if (t1 <= t0) return -INFINITY;
 
@@ -334,17 +348,17 @@ int oracle_max_threads(int nthreads)
 /* Every output: out is [sum(queryLens)][H_q][head_dim] doubles.
  * parts == 0: direct two-pass softmax; parts > 0: split-K with that many
  * partitions per row, merged by log-sum-exp. */
-int oracle_pa_decode(double *out, const uint16_t *q, const void *kc,
+int oracle_pa_decode(double *out, const void *q, const void *kc,
                      const void *vc, const int32_t *block_tables,
                      const int32_t *seq_lens, const int32_t *query_lens,
                      const int32_t *windows, int window, double scale,
                      int batch, int hq, int hkv, int d, int bs, int num_blocks,
                      int max_blocks_per_seq, int kv_fp8, double k_scale, double v_scale,
-                     int parts, int nthreads)
+                     int q_fp8, double q_scale, int parts, int nthreads)
 {
     problem pr = {q, kc, vc, block_tables, seq_lens, query_lens, windows,
                   window, scale, batch, hq, hkv, d, bs, num_blocks,
-                  max_blocks_per_seq, kv_fp8, k_scale, v_scale};
+                  max_blocks_per_seq, kv_fp8, k_scale, v_scale, q_fp8, q_scale};
     if (validate(&pr) || parts < 0) return ORACLE_EINVAL;
     /* list every (b, i, h) with its output slot */
     size_t ntok = 0;
@@ -370,17 +384,18 @@ int oracle_pa_decode(double *out, const uint16_t *q, const void *kc,
 
 /* A chosen subset of outputs: sel is [nsel][3] (b, i, h); out is [nsel][d]. */
 int oracle_pa_decode_select(double *out, const int32_t *sel, int nsel,
-                            const uint16_t *q, const void *kc,
+                            const void *q, const void *kc,
                             const void *vc, const int32_t *block_tables,
                             const int32_t *seq_lens, const int32_t *query_lens,
                             const int32_t *windows, int window, double scale,
                             int batch, int hq, int hkv, int d, int bs,
                             int num_blocks, int max_blocks_per_seq, int kv_fp8,
-                            double k_scale, double v_scale, int nthreads)
+                            double k_scale, double v_scale, int q_fp8,
+                            double q_scale, int nthreads)
 {
     problem pr = {q, kc, vc, block_tables, seq_lens, query_lens, windows,
                   window, scale, batch, hq, hkv, d, bs, num_blocks,
-                  max_blocks_per_seq, kv_fp8, k_scale, v_scale};
+                  max_blocks_per_seq, kv_fp8, k_scale, v_scale, q_fp8, q_scale};
     if (validate(&pr)) return ORACLE_EINVAL;
     for (int j = 0; j < nsel; ++j) {
         int b = sel[3 * j], i = sel[3 * j + 1], h = sel[3 * j + 2];
@@ -398,17 +413,18 @@ int oracle_pa_decode_select(double *out, const int32_t *sel, int nsel,
 
 /* Softmax weights of one query (b, i, h) over every cached position of its
  * row: w is [seq_lens[b]] doubles, zero outside the visible range. */
-int oracle_softmax_weights(double *w, int b, int i, int h, const uint16_t *q,
+int oracle_softmax_weights(double *w, int b, int i, int h, const void *q,
                            const void *kc, const void *vc,
                            const int32_t *block_tables, const int32_t *seq_lens,
                            const int32_t *query_lens, const int32_t *windows,
                            int window, double scale, int batch, int hq, int hkv,
                            int d, int bs, int num_blocks, int max_blocks_per_seq,
-                           int kv_fp8, double k_scale, double v_scale)
+                           int kv_fp8, double k_scale, double v_scale,
+                           int q_fp8, double q_scale)
 {
     problem pr = {q, kc, vc, block_tables, seq_lens, query_lens, windows,
                   window, scale, batch, hq, hkv, d, bs, num_blocks,
-                  max_blocks_per_seq, kv_fp8, k_scale, v_scale};
+                  max_blocks_per_seq, kv_fp8, k_scale, v_scale, q_fp8, q_scale};
     if (validate(&pr)) return ORACLE_EINVAL;
     if (b < 0 || b >= batch || i < 0 || i >= query_lens[b] || h < 0 || h >= hq)
         return ORACLE_EINVAL;

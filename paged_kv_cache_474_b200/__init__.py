@@ -33,6 +33,9 @@ PA_VARIANT_AUTO = 0
 PA_VARIANT_FMA = 1
 PA_VARIANT_MMA = 2
 
+PA_DTYPE_BF16 = 0
+PA_DTYPE_FP8_E4M3 = 1
+
 
 class pa_params(ctypes.Structure):
     _fields_ = [
@@ -50,6 +53,11 @@ class pa_params(ctypes.Structure):
         ("force_variant", ctypes.c_int),
         ("force_partitions", ctypes.c_int),
         ("profile_events", ctypes.c_void_p),
+        ("q_dtype", ctypes.c_int),
+        ("kv_dtype", ctypes.c_int),
+        ("q_scale", ctypes.c_float),
+        ("k_scale", ctypes.c_float),
+        ("v_scale", ctypes.c_float),
     ]
 
 
@@ -204,7 +212,8 @@ def _stream_handle(stream=None):
 def make_params(*, batch, num_q_heads, num_kv_heads, head_dim, num_blocks,
                 max_blocks_per_seq, max_span_hint=0, max_query_len_hint=0,
                 windows=None, workspace=None, force_variant=PA_VARIANT_AUTO,
-                force_partitions=0) -> pa_params:
+                force_partitions=0, q_dtype=PA_DTYPE_BF16, kv_dtype=PA_DTYPE_BF16,
+                q_scale=0.0, k_scale=0.0, v_scale=0.0) -> pa_params:
     p = pa_params()
     p.batch = int(batch)
     p.num_q_heads = int(num_q_heads)
@@ -220,6 +229,11 @@ def make_params(*, batch, num_q_heads, num_kv_heads, head_dim, num_blocks,
         p.workspace_bytes = workspace.numel() * workspace.element_size()
     p.force_variant = int(force_variant)
     p.force_partitions = int(force_partitions)
+    p.q_dtype = int(q_dtype)
+    p.kv_dtype = int(kv_dtype)
+    p.q_scale = float(q_scale)
+    p.k_scale = float(k_scale)
+    p.v_scale = float(v_scale)
     return p
 
 
@@ -251,7 +265,12 @@ def params_for(wl, *, workspace=None, hints=True, force_variant=PA_VARIANT_AUTO,
                        max_span_hint=span, max_query_len_hint=qlen,
                        windows=wl.windows, workspace=workspace,
                        force_variant=force_variant,
-                       force_partitions=force_partitions)
+                       force_partitions=force_partitions,
+                       q_dtype=PA_DTYPE_FP8_E4M3 if wl.q_fp8 else PA_DTYPE_BF16,
+                       kv_dtype=PA_DTYPE_FP8_E4M3 if wl.kv_fp8 else PA_DTYPE_BF16,
+                       q_scale=wl.q_scale if wl.q_fp8 else 0.0,
+                       k_scale=wl.k_scale if wl.kv_fp8 else 0.0,
+                       v_scale=wl.v_scale if wl.kv_fp8 else 0.0)
 
 
 def alloc_workspace(params: pa_params, kv_block_size: int, device="cuda"):
@@ -282,7 +301,7 @@ def decode(wl, *, out=None, workspace=None, hints=True, force_variant=PA_VARIANT
             p.workspace = workspace.data_ptr()
             p.workspace_bytes = workspace.numel()
     if out is None:
-        out = torch.empty_like(wl.q)
+        out = torch.empty(wl.q.shape, dtype=torch.bfloat16, device=wl.q.device)
     _check(pa_decode(out.data_ptr(), wl.q.data_ptr(), wl.k_cache.data_ptr(),
                      wl.v_cache.data_ptr(), wl.block_tables.data_ptr(),
                      wl.seq_lens.data_ptr(), wl.query_lens.data_ptr(), wl.scale,

@@ -108,7 +108,22 @@ int check_params(const pa_params* p, int bs) {
   if (p->force_variant != PA_VARIANT_AUTO && p->force_variant != PA_VARIANT_FMA &&
       p->force_variant != PA_VARIANT_MMA)
     return fail(PA_ERR_ARG, "unknown force_variant %d", p->force_variant);
+  // FP8 operands need their scales (aiter PR #2914 review: validate that
+  // query_scale / key_scale / value_scale are present for FP8 tensors).
+  auto good_scale = [](float x) { return x > 0.f && x <= 3.0e38f; };
+  for (int dt : {p->q_dtype, p->kv_dtype})
+    if (dt != PA_DTYPE_BF16 && dt != PA_DTYPE_FP8_E4M3)
+      return fail(PA_ERR_ARG, "unknown dtype %d (q_dtype / kv_dtype)", dt);
+  if (p->q_dtype == PA_DTYPE_FP8_E4M3 && !good_scale(p->q_scale))
+    return fail(PA_ERR_ARG, "FP8 query needs a finite q_scale > 0 (got %g)", (double)p->q_scale);
+  if (p->kv_dtype == PA_DTYPE_FP8_E4M3 && !(good_scale(p->k_scale) && good_scale(p->v_scale)))
+    return fail(PA_ERR_ARG, "FP8 KV caches need finite k_scale and v_scale > 0 (got %g, %g)",
+                (double)p->k_scale, (double)p->v_scale);
   return PA_OK;
+}
+
+bool any_fp8(const pa_params* p) {
+  return p->q_dtype == PA_DTYPE_FP8_E4M3 || p->kv_dtype == PA_DTYPE_FP8_E4M3;
 }
 
 // Resident CTAs per SM of a kernel instance, queried once per device.
@@ -118,7 +133,7 @@ int cached_occupancy(bool mma, const pa::KernelShape& k, size_t smem) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
   const std::vector<long long> key = {dev, mma, k.head_dim, k.consumer_warps, k.stages, k.n8,
-                                      (long long)smem};
+                                      k.kv_fp8, (long long)smem};
   {
     std::lock_guard<std::mutex> lock(mu);
     auto it = cache.find(key);
@@ -164,7 +179,10 @@ int make_plan(const pa_params* p, int bs, int span, int qlen, int num_sms, int c
     return fail(PA_ERR_UNSUPPORTED, "KV pool rows exceed the tensor map's 32-bit coordinates");
   if (variant == PA_VARIANT_FMA && p->head_dim == 256)
     return fail(PA_ERR_UNSUPPORTED, "head_dim 256 runs on the tensor-core kernel only");
+  if (variant == PA_VARIANT_FMA && any_fp8(p))
+    return fail(PA_ERR_UNSUPPORTED, "FP8 operands run on the tensor-core kernel only");
   const bool mma = variant == PA_VARIANT_MMA;
+  const bool kv8 = p->kv_dtype == PA_DTYPE_FP8_E4M3;
   const int ncw = mma ? 4 : (rmax <= 16 ? 4 : 8);
   // tensor-core warps cover 8 rows (one n-tile) when the unit has <= 8 rows,
   // else 16 (head_dim 256: always 8, its accumulators are twice as wide); a
@@ -175,12 +193,17 @@ int make_plan(const pa_params* p, int bs, int span, int qlen, int num_sms, int c
   const int nslab = (int)cdiv(rmax, slab_rows);
   pl.shape.head_dim = p->head_dim;
   pl.shape.consumer_warps = ncw;
-  pl.shape.stages = p->head_dim == 64 ? 4 : 3;  // 16, 32 or 64 KB per stage
+  pl.shape.kv_fp8 = kv8;
+  // bf16: 16, 32 or 64 KB per stage; FP8: 8, 16 or 32 KB per stage
+  if (!kv8)
+    pl.shape.stages = p->head_dim == 64 ? 4 : 3;
+  else
+    pl.shape.stages = p->head_dim == 64 ? 8 : p->head_dim == 128 ? 4 : 3;
 
   // Partition-size cap: the CTA caches its slice of the block table in smem.
   const int cap = std::max(TS, ((pa::kMaxTableCache - 2) * bs) / TS * TS);
   auto smem_for = [&](int ptok) {
-    return mma ? pa::mma_smem_bytes(p->head_dim, pl.shape.stages, ptok, bs)
+    return mma ? pa::mma_smem_bytes(p->head_dim, kv8 ? 1 : 2, pl.shape.stages, ptok, bs)
                : pa::fma_smem_bytes(p->head_dim, pl.shape.stages, ptok, bs);
   };
   if (num_sms <= 0) {
@@ -265,17 +288,19 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 3-D map of a KV cache viewed as (64 elements, rows, head_dim/64 halves):
-// element stride 1, row stride head_dim*2 bytes, half stride 128 bytes.  A
-// box of (64, box_rows, halves) lands in smem as [half][row][128 B] with the
-// 128-byte swizzle (the half stride is smaller than the row stride on purpose:
-// the box's halves become separate 128-byte-wide tiles).  Encodings are cached
-// per (base, rows, head_dim, box_rows).
-int kv_tensor_map(CUtensorMap* out, const void* base, long long rows, int head_dim, int box_rows) {
+// 3-D map of a KV cache viewed as (box width W bytes, rows, row bytes / W
+// sub-tiles), W = min(row bytes, 128): element stride 1, row stride
+// head_dim * elem_bytes, sub-tile stride W bytes.  A box of (W, box_rows, all
+// sub-tiles) lands in smem as [sub-tile][row][W bytes] with the W-byte
+// swizzle (the sub-tile stride is smaller than the row stride on purpose: the
+// box's sub-tiles become separate W-byte-wide tiles).  Encodings are cached
+// per (base, rows, head_dim, elem_bytes, box_rows).
+int kv_tensor_map(CUtensorMap* out, const void* base, long long rows, int head_dim,
+                  int elem_bytes, int box_rows) {
   struct Entry {
     const void* base;
     long long rows;
-    int d, br;
+    int d, eb, br;
     CUtensorMap map;
   };
   static std::mutex mu;
@@ -283,26 +308,35 @@ int kv_tensor_map(CUtensorMap* out, const void* base, long long rows, int head_d
   {
     std::lock_guard<std::mutex> lock(mu);
     for (const Entry& e : cache)
-      if (e.base == base && e.rows == rows && e.d == head_dim && e.br == box_rows) {
+      if (e.base == base && e.rows == rows && e.d == head_dim && e.eb == elem_bytes &&
+          e.br == box_rows) {
         *out = e.map;
         return PA_OK;
       }
   }
   auto fn = encode_fn();
   if (!fn) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
-  const cuuint64_t dims[3] = {64u, (cuuint64_t)rows, (cuuint64_t)(head_dim / 64)};
-  const cuuint64_t strides[2] = {(cuuint64_t)head_dim * 2, 128u};
-  const cuuint32_t box[3] = {64u, (cuuint32_t)box_rows, (cuuint32_t)(head_dim / 64)};
+  const int row_bytes = head_dim * elem_bytes;
+  const int w = std::min(row_bytes, 128);
+  const cuuint64_t dims[3] = {(cuuint64_t)(w / elem_bytes), (cuuint64_t)rows,
+                              (cuuint64_t)(row_bytes / w)};
+  const cuuint64_t strides[2] = {(cuuint64_t)row_bytes, (cuuint64_t)w};
+  const cuuint32_t box[3] = {(cuuint32_t)(w / elem_bytes), (cuuint32_t)box_rows,
+                             (cuuint32_t)(row_bytes / w)};
   const cuuint32_t estr[3] = {1u, 1u, 1u};
   Entry e;
   e.base = base;
   e.rows = rows;
   e.d = head_dim;
+  e.eb = elem_bytes;
   e.br = box_rows;
-  const CUresult r = fn(&e.map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
-                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUresult r = fn(&e.map,
+                        elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                        : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                        3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        w == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(PA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   std::lock_guard<std::mutex> lock(mu);
   if (cache.size() >= 16) cache.erase(cache.begin());
@@ -364,8 +398,9 @@ int decode_impl(void* dst, const void* q, const void* kCache, const void* vCache
   pa::DecodeArgs a;
   memset(&a, 0, sizeof a);
   a.q = static_cast<const __nv_bfloat16*>(q);
-  a.k_cache = static_cast<const __nv_bfloat16*>(kCache);
-  a.v_cache = static_cast<const __nv_bfloat16*>(vCache);
+  a.q8 = static_cast<const uint8_t*>(q);
+  a.k_cache = kCache;
+  a.v_cache = vCache;
   a.block_tables = blockTables;
   a.seq_lens = seqLens;
   a.query_lens = queryLens;
@@ -376,7 +411,13 @@ int decode_impl(void* dst, const void* q, const void* kCache, const void* vCache
     a.ws_lse = reinterpret_cast<float*>(ws);
     a.ws_o = reinterpret_cast<float*>(ws + pl.lse_bytes);
   }
-  a.scale_log2 = scale * 1.4426950408889634f;
+  // FP8 scales: q_scale * k_scale multiplies every score, v_scale every output
+  double sc = (double)scale * 1.4426950408889634;
+  if (p->q_dtype == PA_DTYPE_FP8_E4M3) sc *= p->q_scale;
+  if (p->kv_dtype == PA_DTYPE_FP8_E4M3) sc *= p->k_scale;
+  a.scale_log2 = (float)sc;
+  a.v_scale = p->kv_dtype == PA_DTYPE_FP8_E4M3 ? p->v_scale : 1.f;
+  a.q_fp8 = p->q_dtype == PA_DTYPE_FP8_E4M3;
   a.window = window;
   a.batch = p->batch;
   a.num_q_heads = p->num_q_heads;
@@ -405,8 +446,9 @@ int decode_impl(void* dst, const void* q, const void* kCache, const void* vCache
       CUtensorMap tk, tv;
       const long long rows = (long long)p->num_blocks * p->num_kv_heads * bs;
       const int br = std::min(bs, TS);
-      rc = kv_tensor_map(&tk, kCache, rows, p->head_dim, br);
-      if (!rc) rc = kv_tensor_map(&tv, vCache, rows, p->head_dim, br);
+      const int eb = p->kv_dtype == PA_DTYPE_FP8_E4M3 ? 1 : 2;
+      rc = kv_tensor_map(&tk, kCache, rows, p->head_dim, eb, br);
+      if (!rc) rc = kv_tensor_map(&tv, vCache, rows, p->head_dim, eb, br);
       if (rc) return rc;
       e = pa::launch_partition_mma(a, pl.shape, tk, tv, grid, in.smem_bytes, stream);
     } else {
@@ -521,8 +563,10 @@ size_t pa_host_workspace_size(const pa_params* params, int kvBlockSize, int wind
                    &qlen, &ntok))
     return (size_t)-1;
   const size_t B = params->batch;
-  const size_t qbytes = align256((size_t)ntok * params->num_q_heads * params->head_dim * 2);
-  size_t total = 2 * qbytes + align256(B * params->max_blocks_per_seq * 4) + 3 * align256(B * 4);
+  const size_t rowe = (size_t)ntok * params->num_q_heads * params->head_dim;
+  const size_t qbytes = align256(rowe * (params->q_dtype == PA_DTYPE_FP8_E4M3 ? 1 : 2));
+  size_t total = qbytes + align256(rowe * 2) + align256(B * params->max_blocks_per_seq * 4) +
+                 3 * align256(B * 4);
   if (qlen > 0) {
     Plan pl;
     if (make_plan(params, kvBlockSize, span, qlen, 0, 0, &pl)) return (size_t)-1;
@@ -560,12 +604,13 @@ int pa_decode_host(void* dst_host, const void* q_host, const void* kCache, const
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* ws = static_cast<char*>(params->workspace);
-  const size_t qbytes_raw = (size_t)ntok * params->num_q_heads * params->head_dim * 2;
-  const size_t qbytes = align256(qbytes_raw);
+  const size_t rowe = (size_t)ntok * params->num_q_heads * params->head_dim;
+  const size_t qbytes_raw = rowe * (params->q_dtype == PA_DTYPE_FP8_E4M3 ? 1 : 2);
+  const size_t dbytes_raw = rowe * 2;
   const size_t btbytes = (size_t)B * params->max_blocks_per_seq * 4;
   char* d_q = ws;
-  char* d_dst = d_q + qbytes;
-  char* d_bt = d_dst + qbytes;
+  char* d_dst = d_q + align256(qbytes_raw);
+  char* d_bt = d_dst + align256(dbytes_raw);
   char* d_S = d_bt + align256(btbytes);
   char* d_L = d_S + align256((size_t)B * 4);
   char* d_W = d_L + align256((size_t)B * 4);
@@ -592,7 +637,7 @@ int pa_decode_host(void* dst_host, const void* q_host, const void* kCache, const
                      scale, window, kvBlockSize, &dp, st, span, qlen);
     if (rc) return rc;
   }
-  if (qbytes_raw) e = cudaMemcpyAsync(dst_host, d_dst, qbytes_raw, cudaMemcpyDeviceToHost, st);
+  if (dbytes_raw) e = cudaMemcpyAsync(dst_host, d_dst, dbytes_raw, cudaMemcpyDeviceToHost, st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return fail(PA_ERR_CUDA, "device-to-host copy: %s", cudaGetErrorString(e));
   return succeed();

@@ -179,7 +179,7 @@ __global__ void __launch_bounds__(32 * (NCW + 1), (NCW <= 4 ? 2 : 1))
           const size_t off =
               (((size_t)phys * a.num_kv_heads + kvh) * a.block_size + (t_a - (jj << a.block_shift))) *
               (size_t)D;
-          src = (isv ? a.v_cache : a.k_cache) + off;
+          src = static_cast<const __nv_bfloat16*>(isv ? a.v_cache : a.k_cache) + off;
           dsto = s * T::STAGE_BYTES + (isv ? TS * T::ROWB : 0) + (t_a - c0) * T::ROWB;
         }
       }
@@ -415,12 +415,25 @@ __global__ void __launch_bounds__(32 * (NCW + 1), (NCW <= 4 ? 2 : 1))
 // holds, so the online-softmax rescale needs no data movement.  Tokens a box
 // brings in from outside the row's visible union get score -inf and their V
 // lanes are zeroed in registers, so uninitialised cache slots never reach O.
+//
+// FP8 e4m3 caches (F8): a token row is D bytes, staged the same way, and the
+// MMAs run on f16 operands (e4m3 -> f16 is exact, one cvt per code pair; Q is
+// converted to f16 once, P is packed as f16).  The reduction order over d and
+// the order of O^T's rows are free, so the fragments are chosen to suit
+// byte-wide data: a k-step takes one 16-byte chunk (16 dims); the thread
+// that ldmatrix gives bytes 4c..4c+3 of a token row uses them as MMA k
+// indices 2c, 2c+1, 2c+8, 2c+9, and Q^T is loaded with the same map.  For
+// V^T, ldmatrix.trans over b16 pairs gives a thread two dims (2g, 2g+1) of
+// two tokens; one byte permute regroups them by dim, so O^T row g of the
+// tile is dim 2g and row g+8 is dim 2g+1.  q_scale * k_scale is folded into
+// the score scale and v_scale into the output normalisation.
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, bool F8>
 struct MmaTraits {
-  static constexpr int HALVES = D / 64;
-  static constexpr int HALF_BYTES = TS * 128;
-  static constexpr int KV_BYTES = HALVES * HALF_BYTES;
+  static constexpr int ROW_BYTES = F8 ? D : 2 * D;                  // one token of one kv head
+  static constexpr int BOXW = ROW_BYTES < 128 ? ROW_BYTES : 128;    // swizzle span of a box row
+  static constexpr int HALVES = ROW_BYTES / BOXW;                   // box sub-tiles along d
+  static constexpr int KV_BYTES = TS * ROW_BYTES;
   static constexpr int STAGE_BYTES = 2 * KV_BYTES;
   static constexpr int KSTEPS = D / 16;  // 16-wide reduction steps over d
   static constexpr int MD = D / 16;      // 16-dim M tiles of O^T
@@ -436,11 +449,17 @@ struct MmaCombine {
   static constexpr int BYTES = (ACC_FLOATS + L_FLOATS + M_FLOATS) * 4;
 };
 
-// Byte offset, within a box, of 16-byte chunk `chunk` (0 .. D/8-1) of row lt
-// (lt < 16, relative to a 16-row aligned chunk start): half (chunk / 8) of the
-// box, row lt, chunk position swizzled by the row's low three bits.
+// Byte offset, within a box, of 16-byte chunk `chunk` of row lt (lt < 16,
+// relative to a 16-row aligned chunk start).  128-byte box rows: half
+// (chunk / 8) of the box, row lt, chunk position swizzled by the row's low
+// three bits.  64-byte box rows (FP8, head_dim 64; 64-byte swizzle): chunk
+// position swizzled by bits 1..2 of the row.
+template <int BOXW>
 __device__ __forceinline__ uint32_t box_off(int lt, int chunk, int BR) {
-  return (uint32_t)((chunk >> 3) * BR * 128 + lt * 128 + (((chunk & 7) ^ (lt & 7)) << 4));
+  if constexpr (BOXW == 128)
+    return (uint32_t)((chunk >> 3) * BR * 128 + lt * 128 + (((chunk & 7) ^ (lt & 7)) << 4));
+  else
+    return (uint32_t)(lt * 64 + (((chunk & 3) ^ ((lt >> 1) & 3)) << 4));
 }
 
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
@@ -452,12 +471,12 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
 // Register caps keep 4 (one n-tile) or 3 (two n-tiles) warps per SM
 // sub-partition, so two CTAs fit per SM; head_dim 256 runs one CTA per SM
 // (its 192 KB ring) and takes the larger cap for its wider accumulators.
-template <int D, int NCW, int NSTAGE, int N8>
+template <int D, int NCW, int NSTAGE, int N8, bool F8>
 __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
     pa_partition_mma_kernel(const __grid_constant__ DecodeArgs a,
                             const __grid_constant__ CUtensorMap tmk,
                             const __grid_constant__ CUtensorMap tmv) {
-  using T = MmaTraits<D>;
+  using T = MmaTraits<D, F8>;
   using C = MmaCombine<D, NCW, N8>;
   constexpr int RT = C::RT;
   static_assert(C::BYTES <= NSTAGE * T::STAGE_BYTES, "combine area must fit in the ring");
@@ -538,9 +557,9 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
   float* comb_m = comb_l + C::L_FLOATS;
   const int NRT = (Rs + RT - 1) / RT;  // row tiles in this slab
 
-  // A box is BR token rows of one (block, kv head): [D/64 halves][BR rows][128 B].
+  // A box is BR token rows of one (block, kv head): [halves][BR rows][BOXW bytes].
   const int BR = min(a.block_size, TS);
-  const uint32_t box_bytes = (uint32_t)BR * 128u * T::HALVES;
+  const uint32_t box_bytes = (uint32_t)BR * T::ROW_BYTES;
   int qoff = 0;
 
   if (warp == 0) {
@@ -613,13 +632,16 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
     // lane parts of the ldmatrix row addresses (token row within the chunk,
     // 16-byte chunk parity) for K (A operand) and V (A operand, transposed)
     const int lt_k = (((lane >> 3) & 1) << 3) + (lane & 7), ck_k = lane >> 4;
-    const int lt_v = ((lane >> 4) << 3) + (lane & 7), ck_v = (lane >> 3) & 1;
+    // (FP8 V uses the K addresses: its x4 covers tokens 0-7 / 8-15 of two chunks.)
+    const int lt_v = F8 ? lt_k : ((lane >> 4) << 3) + (lane & 7);
+    const int ck_v = F8 ? ck_k : (lane >> 3) & 1;
     int lo_max, hi_min, dummy;
     query_range(S, L, L - 1, w, lo_max, dummy);  // the last token sees the latest start
     query_range(S, L, 0, w, dummy, hi_min);      // the first token sees the earliest end
 
-    // Q^T as B fragments (exact bf16): n-tile n holds warp-tile rows n*8..n*8+7;
-    // this thread feeds row n*8 + quad, dims ks*16 + 2*qi (+1) and +8 (+9).
+    // Q^T as B fragments: n-tile n holds warp-tile rows n*8..n*8+7; this
+    // thread feeds row n*8 + quad, dims ks*16 + 2*qi (+1) and +8 (+9) (bf16
+    // caches), or dims ks*16 + 4*qi .. +3 (FP8 caches, f16 operands).
     uint32_t qb[T::KSTEPS][N8][2];
     // Softmax statistics of the rows n*8 + 2*qi + j (j = 0, 1): the O^T columns
     // this thread accumulates.
@@ -627,17 +649,41 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
 #pragma unroll
     for (int n = 0; n < N8; ++n) {
       const int rq = rt * RT + n * 8 + quad;
-      const uint32_t* qp = nullptr;
-      if (rq < Rs) {
+      size_t qrow = 0;
+      const bool has_q = rq < Rs;
+      if (has_q) {
         const int rr = row0 + rq;
         const int i = rr / a.group, j = rr - (rr / a.group) * a.group;
-        qp = reinterpret_cast<const uint32_t*>(
-            a.q + ((size_t)(qoff + i) * a.num_q_heads + (size_t)kvh * a.group + j) * D);
+        qrow = ((size_t)(qoff + i) * a.num_q_heads + (size_t)kvh * a.group + j) * D;
       }
 #pragma unroll
       for (int ks = 0; ks < T::KSTEPS; ++ks) {
-        qb[ks][n][0] = qp ? __ldg(qp + ks * 8 + qi) : 0u;
-        qb[ks][n][1] = qp ? __ldg(qp + ks * 8 + qi + 4) : 0u;
+        uint32_t b0 = 0u, b1 = 0u;
+        if (has_q) {
+          if constexpr (F8) {
+            if (a.q_fp8) {
+              const uint32_t w4 = __ldg(reinterpret_cast<const uint32_t*>(a.q8 + qrow) + ks * 4 + qi);
+              b0 = e4m3x2_to_f16x2(w4 & 0xffffu);
+              b1 = e4m3x2_to_f16x2(w4 >> 16);
+            } else {
+              const uint2 w4 = __ldg(reinterpret_cast<const uint2*>(a.q + qrow) + ks * 4 + qi);
+              b0 = bf16x2_to_f16x2(w4.x);
+              b1 = bf16x2_to_f16x2(w4.y);
+            }
+          } else {
+            if (a.q_fp8) {
+              const unsigned short* qp = reinterpret_cast<const unsigned short*>(a.q8 + qrow);
+              b0 = f16x2_to_bf16x2(e4m3x2_to_f16x2(__ldg(qp + ks * 8 + qi)));
+              b1 = f16x2_to_bf16x2(e4m3x2_to_f16x2(__ldg(qp + ks * 8 + qi + 4)));
+            } else {
+              const uint32_t* qp = reinterpret_cast<const uint32_t*>(a.q + qrow);
+              b0 = __ldg(qp + ks * 8 + qi);
+              b1 = __ldg(qp + ks * 8 + qi + 4);
+            }
+          }
+        }
+        qb[ks][n][0] = b0;
+        qb[ks][n][1] = b1;
       }
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
@@ -670,7 +716,7 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
       for (int ch = slice; ch < TS / 16; ch += nslice) {
         const int tb = ch * 16;
         // the chunk's 16 tokens lie in one box (BR >= 16)
-        const uint32_t cbase = (uint32_t)((tb >> brs) * box_bytes + (tb & (BR - 1)) * 128);
+        const uint32_t cbase = (uint32_t)((tb >> brs) * box_bytes + (tb & (BR - 1)) * T::BOXW);
         // S^T = K Q^T; with one n-tile, two accumulator sets (even / odd d
         // steps) halve the dependent MMA chain.
         constexpr int NACC = N8 == 1 ? 2 : 1;
@@ -679,13 +725,34 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
         for (int u = 0; u < 2; ++u)
 #pragma unroll
           for (int n = 0; n < N8; ++n) sc[u][n][0] = sc[u][n][1] = sc[u][n][2] = sc[u][n][3] = 0.f;
+        if constexpr (F8) {
+          // one x4 = tokens 0-7 / 8-15 of chunks 2kp, 2kp+1: two k-steps
 #pragma unroll
-        for (int ks = 0; ks < T::KSTEPS; ++ks) {
-          uint32_t ka[4];
-          ldsm_x4(Ks + cbase + box_off(lt_k, ks * 2 + ck_k, BR), ka[0], ka[1], ka[2], ka[3]);
+          for (int kp = 0; kp < T::KSTEPS / 2; ++kp) {
+            uint32_t r[4];
+            ldsm_x4(Ks + cbase + box_off<T::BOXW>(lt_k, kp * 2 + ck_k, BR), r[0], r[1], r[2], r[3]);
 #pragma unroll
-          for (int n = 0; n < N8; ++n)
-            mma_bf16_16816(sc[ks % NACC][n], ka, qb[ks][n][0], qb[ks][n][1]);
+            for (int h = 0; h < 2; ++h) {
+              const uint32_t ka[4] = {e4m3x2_to_f16x2(r[2 * h] & 0xffffu),
+                                      e4m3x2_to_f16x2(r[2 * h + 1] & 0xffffu),
+                                      e4m3x2_to_f16x2(r[2 * h] >> 16),
+                                      e4m3x2_to_f16x2(r[2 * h + 1] >> 16)};
+              const int ks = 2 * kp + h;
+#pragma unroll
+              for (int n = 0; n < N8; ++n)
+                mma_f16_16816(sc[ks % NACC][n], ka, qb[ks][n][0], qb[ks][n][1]);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int ks = 0; ks < T::KSTEPS; ++ks) {
+            uint32_t ka[4];
+            ldsm_x4(Ks + cbase + box_off<T::BOXW>(lt_k, ks * 2 + ck_k, BR), ka[0], ka[1], ka[2],
+                    ka[3]);
+#pragma unroll
+            for (int n = 0; n < N8; ++n)
+              mma_bf16_16816(sc[ks % NACC][n], ka, qb[ks][n][0], qb[ks][n][1]);
+          }
         }
         // element e of n-tile n: token tb + quad + 8*(e>>1), row n*8 + 2*qi + (e&1)
         float p[N8][4];
@@ -734,8 +801,13 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
         uint32_t pb[N8][2];
 #pragma unroll
         for (int n = 0; n < N8; ++n) {
-          pb[n][0] = movmatrix_trans(pack_bf16x2(p[n][0], p[n][1]));
-          pb[n][1] = movmatrix_trans(pack_bf16x2(p[n][2], p[n][3]));
+          if constexpr (F8) {
+            pb[n][0] = movmatrix_trans(pack_f16x2(p[n][0], p[n][1]));
+            pb[n][1] = movmatrix_trans(pack_f16x2(p[n][2], p[n][3]));
+          } else {
+            pb[n][0] = movmatrix_trans(pack_bf16x2(p[n][0], p[n][1]));
+            pb[n][1] = movmatrix_trans(pack_bf16x2(p[n][2], p[n][3]));
+          }
         }
         uint32_t mk_lo = 0xffffffffu, mk_hi = 0xffffffffu;
         if (boundary) {
@@ -744,16 +816,41 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
           mk_lo = (in(t) ? 0x0000ffffu : 0u) | (in(t + 1) ? 0xffff0000u : 0u);
           mk_hi = (in(t + 8) ? 0x0000ffffu : 0u) | (in(t + 9) ? 0xffff0000u : 0u);
         }
+        if constexpr (F8) {
+          // one x4.trans = tokens 0-7 / 8-15 of chunks 2mp, 2mp+1: two M tiles;
+          // a register holds dims (2g, 2g+1) of tokens (2c, 2c+1), regrouped
+          // by dim before the conversion (the masks act on converted halves)
 #pragma unroll
-        for (int md = 0; md < T::MD; ++md) {
-          uint32_t va[4];
-          ldsm_x4_t(Vs + cbase + box_off(lt_v, md * 2 + ck_v, BR), va[0], va[1], va[2], va[3]);
-          va[0] &= mk_lo;
-          va[1] &= mk_lo;
-          va[2] &= mk_hi;
-          va[3] &= mk_hi;
+          for (int mp = 0; mp < T::MD / 2; ++mp) {
+            uint32_t r[4];
+            ldsm_x4_t(Vs + cbase + box_off<T::BOXW>(lt_v, mp * 2 + ck_v, BR), r[0], r[1], r[2],
+                      r[3]);
 #pragma unroll
-          for (int n = 0; n < N8; ++n) mma_bf16_16816(o[md][n], va, pb[n][0], pb[n][1]);
+            for (int h = 0; h < 2; ++h) {
+              const uint32_t t0 = __byte_perm(r[2 * h], 0, 0x3120);
+              const uint32_t t1 = __byte_perm(r[2 * h + 1], 0, 0x3120);
+              const uint32_t va[4] = {e4m3x2_to_f16x2(t0 & 0xffffu) & mk_lo,
+                                      e4m3x2_to_f16x2(t0 >> 16) & mk_lo,
+                                      e4m3x2_to_f16x2(t1 & 0xffffu) & mk_hi,
+                                      e4m3x2_to_f16x2(t1 >> 16) & mk_hi};
+#pragma unroll
+              for (int n = 0; n < N8; ++n)
+                mma_f16_16816(o[2 * mp + h][n], va, pb[n][0], pb[n][1]);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int md = 0; md < T::MD; ++md) {
+            uint32_t va[4];
+            ldsm_x4_t(Vs + cbase + box_off<T::BOXW>(lt_v, md * 2 + ck_v, BR), va[0], va[1], va[2],
+                      va[3]);
+            va[0] &= mk_lo;
+            va[1] &= mk_lo;
+            va[2] &= mk_hi;
+            va[3] &= mk_hi;
+#pragma unroll
+            for (int n = 0; n < N8; ++n) mma_bf16_16816(o[md][n], va, pb[n][0], pb[n][1]);
+          }
         }
       }
       __syncwarp();
@@ -761,15 +858,28 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
     }
 
     named_bar_sync(1, NCW * 32);
-    // O^T element (md, n, e): dim md*16 + quad + 8*(e>>1), row n*8 + 2*qi + (e&1)
+    if constexpr (F8) {
+      // O^T element (md, n, e): dim md*16 + 2*quad + (e>>1), row n*8 + 2*qi + (e&1)
 #pragma unroll
-    for (int md = 0; md < T::MD; ++md)
+      for (int md = 0; md < T::MD; ++md)
 #pragma unroll
-      for (int n = 0; n < N8; ++n)
+        for (int n = 0; n < N8; ++n)
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          comb_acc[(cw * RT + n * 8 + 2 * qi + (e & 1)) * C::LD + md * 16 + quad + ((e >> 1) << 3)] =
-              o[md][n][e];
+          for (int j = 0; j < 2; ++j)
+            *reinterpret_cast<float2*>(
+                &comb_acc[(cw * RT + n * 8 + 2 * qi + j) * C::LD + md * 16 + 2 * quad]) =
+                make_float2(o[md][n][j], o[md][n][j + 2]);
+    } else {
+      // O^T element (md, n, e): dim md*16 + quad + 8*(e>>1), row n*8 + 2*qi + (e&1)
+#pragma unroll
+      for (int md = 0; md < T::MD; ++md)
+#pragma unroll
+        for (int n = 0; n < N8; ++n)
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            comb_acc[(cw * RT + n * 8 + 2 * qi + (e & 1)) * C::LD + md * 16 + quad +
+                     ((e >> 1) << 3)] = o[md][n][e];
+    }
 #pragma unroll
     for (int n = 0; n < N8; ++n)
 #pragma unroll
@@ -820,14 +930,14 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
     const float Z = s_rowz[r];
     const int rr = row0 + r;
     if (nparts == 1) {
-      const float inv = 1.f / Z;
+      const float inv = a.v_scale / Z;
       const int i = rr / a.group, j = rr - (rr / a.group) * a.group;
       __nv_bfloat16* dp =
           a.dst + ((size_t)(qoff + i) * a.num_q_heads + (size_t)kvh * a.group + j) * D + c4 * 4;
       *reinterpret_cast<__nv_bfloat162*>(dp) = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
       *reinterpret_cast<__nv_bfloat162*>(dp + 2) = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
     } else {
-      const float inv = Z > 0.f ? 1.f / Z : 0.f;
+      const float inv = Z > 0.f ? a.v_scale / Z : 0.f;
       const size_t base =
           ((size_t)(b * a.num_kv_heads + kvh) * a.max_parts + part) * a.max_rows + rr;
       *reinterpret_cast<float4*>(a.ws_o + base * D + c4 * 4) =
@@ -1086,10 +1196,10 @@ int occupancy_fma_t(size_t smem) {
   return n;
 }
 
-template <int D, int NCW, int NSTAGE, int N8>
+template <int D, int NCW, int NSTAGE, int N8, bool F8>
 cudaError_t launch_mma_t(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
                          dim3 grid, size_t smem, cudaStream_t stream) {
-  auto kern = pa_partition_mma_kernel<D, NCW, NSTAGE, N8>;
+  auto kern = pa_partition_mma_kernel<D, NCW, NSTAGE, N8, F8>;
   cudaError_t e = ensure_smem_attrs(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   // Programmatic stream serialization: CTAs may start (and set up their
@@ -1108,9 +1218,9 @@ cudaError_t launch_mma_t(const DecodeArgs& a, const CUtensorMap& tk, const CUten
   return cudaLaunchKernelEx(&cfg, kern, a, tk, tv);
 }
 
-template <int D, int NCW, int NSTAGE, int N8>
+template <int D, int NCW, int NSTAGE, int N8, bool F8>
 int occupancy_mma_t(size_t smem) {
-  auto kern = pa_partition_mma_kernel<D, NCW, NSTAGE, N8>;
+  auto kern = pa_partition_mma_kernel<D, NCW, NSTAGE, N8, F8>;
   if (ensure_smem_attrs(reinterpret_cast<const void*>(kern), smem) != cudaSuccess) return 0;
   int n = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 32 * (NCW + 1), smem) != cudaSuccess)
@@ -1120,35 +1230,48 @@ int occupancy_mma_t(size_t smem) {
 
 }  // namespace
 
-size_t mma_smem_bytes(int head_dim, int stages, int part_tokens, int block_size) {
-  const size_t ring = (size_t)stages * 2 * TS * head_dim * 2;
+size_t mma_smem_bytes(int head_dim, int elem_bytes, int stages, int part_tokens, int block_size) {
+  const size_t ring = (size_t)stages * 2 * TS * head_dim * elem_bytes;
   const size_t nbt = (size_t)part_tokens / block_size + 2;
   return 1024 + ring + 2 * (size_t)stages * sizeof(uint64_t) + nbt * sizeof(int);
 }
 
-#define PA_MMA_DISPATCH(CALL)                                            \
-  if (k.head_dim == 128 && k.consumer_warps == 4 && k.stages == 3 && k.n8 == 1) \
-    CALL(128, 4, 3, 1);                                                  \
-  if (k.head_dim == 128 && k.consumer_warps == 4 && k.stages == 3 && k.n8 == 2) \
-    CALL(128, 4, 3, 2);                                                  \
-  if (k.head_dim == 64 && k.consumer_warps == 4 && k.stages == 4 && k.n8 == 1)  \
-    CALL(64, 4, 4, 1);                                                   \
-  if (k.head_dim == 64 && k.consumer_warps == 4 && k.stages == 4 && k.n8 == 2)  \
-    CALL(64, 4, 4, 2);                                                   \
-  if (k.head_dim == 256 && k.consumer_warps == 4 && k.stages == 3 && k.n8 == 1) \
-    CALL(256, 4, 3, 1);
+// (head_dim, compute warps, stages, n-tiles, FP8 caches).  Rings: bf16 64,
+// 96 and 192 KB for head_dim 64, 128 and 256; FP8 64 KB (head_dim 64, 128:
+// three CTAs per SM fit at 128) and 96 KB (256: two CTAs per SM).
+#define PA_MMA_DISPATCH(CALL)                                                       \
+  if (k.head_dim == 128 && k.consumer_warps == 4 && k.stages == 3 && k.n8 == 1 && !k.kv_fp8) \
+    CALL(128, 4, 3, 1, false);                                                      \
+  if (k.head_dim == 128 && k.consumer_warps == 4 && k.stages == 3 && k.n8 == 2 && !k.kv_fp8) \
+    CALL(128, 4, 3, 2, false);                                                      \
+  if (k.head_dim == 64 && k.consumer_warps == 4 && k.stages == 4 && k.n8 == 1 && !k.kv_fp8)  \
+    CALL(64, 4, 4, 1, false);                                                       \
+  if (k.head_dim == 64 && k.consumer_warps == 4 && k.stages == 4 && k.n8 == 2 && !k.kv_fp8)  \
+    CALL(64, 4, 4, 2, false);                                                       \
+  if (k.head_dim == 256 && k.consumer_warps == 4 && k.stages == 3 && k.n8 == 1 && !k.kv_fp8) \
+    CALL(256, 4, 3, 1, false);                                                      \
+  if (k.head_dim == 128 && k.consumer_warps == 4 && k.stages == 4 && k.n8 == 1 && k.kv_fp8)  \
+    CALL(128, 4, 4, 1, true);                                                       \
+  if (k.head_dim == 128 && k.consumer_warps == 4 && k.stages == 4 && k.n8 == 2 && k.kv_fp8)  \
+    CALL(128, 4, 4, 2, true);                                                       \
+  if (k.head_dim == 64 && k.consumer_warps == 4 && k.stages == 8 && k.n8 == 1 && k.kv_fp8)   \
+    CALL(64, 4, 8, 1, true);                                                        \
+  if (k.head_dim == 64 && k.consumer_warps == 4 && k.stages == 8 && k.n8 == 2 && k.kv_fp8)   \
+    CALL(64, 4, 8, 2, true);                                                        \
+  if (k.head_dim == 256 && k.consumer_warps == 4 && k.stages == 3 && k.n8 == 1 && k.kv_fp8)  \
+    CALL(256, 4, 3, 1, true);
 
 cudaError_t launch_partition_mma(const DecodeArgs& a, const KernelShape& k, const CUtensorMap& tk,
                                  const CUtensorMap& tv, dim3 grid, size_t smem,
                                  cudaStream_t stream) {
-#define PA_CALL(D, N, S, N8) return launch_mma_t<D, N, S, N8>(a, tk, tv, grid, smem, stream)
+#define PA_CALL(D, N, S, N8, F8) return launch_mma_t<D, N, S, N8, F8>(a, tk, tv, grid, smem, stream)
   PA_MMA_DISPATCH(PA_CALL)
 #undef PA_CALL
   return cudaErrorInvalidValue;
 }
 
 int occupancy_partition_mma(const KernelShape& k, size_t smem) {
-#define PA_CALL(D, N, S, N8) return occupancy_mma_t<D, N, S, N8>(smem)
+#define PA_CALL(D, N, S, N8, F8) return occupancy_mma_t<D, N, S, N8, F8>(smem)
   PA_MMA_DISPATCH(PA_CALL)
 #undef PA_CALL
   return 0;

@@ -15,9 +15,10 @@ constexpr int kMaxTableCache = 1024;  // block-table entries a CTA caches in sme
 
 // Everything a decode launch needs; passed by value as a __grid_constant__.
 struct DecodeArgs {
-  const __nv_bfloat16* q;
-  const __nv_bfloat16* k_cache;
-  const __nv_bfloat16* v_cache;
+  const __nv_bfloat16* q;  // bf16 queries (q_fp8 == 0)
+  const uint8_t* q8;       // FP8 e4m3 query codes (q_fp8 == 1)
+  const void* k_cache;     // bf16, or FP8 e4m3 codes (tensor-core kernel only)
+  const void* v_cache;
   const int32_t* block_tables;
   const int32_t* seq_lens;
   const int32_t* query_lens;
@@ -25,7 +26,9 @@ struct DecodeArgs {
   __nv_bfloat16* dst;
   float* ws_lse;  // [B][H_kv][max_parts][max_rows]  log2-domain lse of each partial
   float* ws_o;    // [B][H_kv][max_parts][max_rows][D] normalised partial outputs
-  float scale_log2;  // scale * log2(e): scores are kept in the log2 domain
+  float scale_log2;  // scale * log2(e) (* q_scale * k_scale for FP8 operands): log2-domain scores
+  float v_scale;     // multiplies every output (FP8 V), 1 otherwise
+  int q_fp8;
   int window;
   int batch, num_q_heads, num_kv_heads, group, head_dim;
   int block_size, block_shift, max_blocks_per_seq, num_blocks;
@@ -42,6 +45,7 @@ struct KernelShape {
   int consumer_warps;
   int stages;
   int n8;  // tensor-core variant: 8-row n-tiles per compute warp (1 or 2)
+  int kv_fp8;  // tensor-core variant: FP8 e4m3 K/V caches
 };
 
 // Dynamic shared memory of the FMA partition kernel.
@@ -55,11 +59,12 @@ cudaError_t launch_partition_fma(const DecodeArgs& a, const KernelShape& k, dim3
 int occupancy_partition_fma(const KernelShape& k, size_t smem);
 
 // Dynamic shared memory of the tensor-core partition kernel.
-size_t mma_smem_bytes(int head_dim, int stages, int part_tokens, int block_size);
+size_t mma_smem_bytes(int head_dim, int elem_bytes, int stages, int part_tokens, int block_size);
 
-// Launches the tensor-core partition kernel; tk / tv are 2-D tiled maps of
-// the K and V caches viewed as [rows][head_dim] with 64 x box-rows boxes and
-// the 128-byte swizzle.
+// Launches the tensor-core partition kernel; tk / tv are 3-D tiled maps of
+// the K and V caches: (box width, rows, row bytes / box width) with boxes of
+// (box width, box rows, all) and the 128-byte swizzle (64-byte for the
+// 64-byte rows of FP8 head_dim 64); box width = min(row bytes, 128) bytes.
 cudaError_t launch_partition_mma(const DecodeArgs& a, const KernelShape& k, const CUtensorMap& tk,
                                  const CUtensorMap& tv, dim3 grid, size_t smem,
                                  cudaStream_t stream);

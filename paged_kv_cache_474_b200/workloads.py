@@ -26,7 +26,8 @@ Values are drawn as float32 (uniform(-1,1) for the tiny workload, standard
 normal otherwise) on the requested device and rounded to bf16 (round to
 nearest even); both sides then read the same bf16 bytes.  FP8 caches
 (kv_dtype="fp8_e4m3") quantise those bf16 values per tensor: scale =
-max|x| / 448, codes = round-to-nearest e4m3 of x / scale.
+max|x| / 448, codes = round-to-nearest e4m3 of x / scale; FP8 queries
+(q_dtype="fp8_e4m3") are quantised the same way.
 """
 from __future__ import annotations
 
@@ -64,10 +65,16 @@ class Workload:
     # value is its e4m3 number times k_scale / v_scale.  1.0 for bf16 caches.
     k_scale: float = 1.0
     v_scale: float = 1.0
+    # FP8 queries: q holds e4m3 codes (torch.uint8) whose value is times q_scale
+    q_scale: float = 1.0
 
     @property
     def kv_fp8(self) -> bool:
         return self.k_cache.dtype == torch.uint8
+
+    @property
+    def q_fp8(self) -> bool:
+        return self.q.dtype == torch.uint8
 
     @property
     def batch(self) -> int:
@@ -155,7 +162,12 @@ def to_e4m3(x: torch.Tensor):
     float8_e4m3fn cast rounds to nearest."""
     amax = float(x.abs().max()) if x.numel() else 1.0
     s = (amax / 448.0) if amax > 0 else 1.0
-    codes = (x.float() / s).to(torch.float8_e4m3fn).view(torch.uint8)
+    codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    per_row = int(np.prod(x.shape[1:])) if x.dim() > 1 else 1
+    step = max(1, (1 << 28) // max(per_row, 1))  # float32 staging under 1 GiB
+    for a in range(0, max(x.shape[0], 0), step):
+        b = min(x.shape[0], a + step)
+        codes[a:b] = (x[a:b].float() / s).to(torch.float8_e4m3fn).view(torch.uint8)
     return codes, s
 
 
@@ -166,7 +178,7 @@ def make_workload(*, seq_lens: Sequence[int], query_lens: Sequence[int],
                   scale: Optional[float] = None, dist: str = "normal",
                   seed: int = 0, device="cpu", spare_blocks: int = 1,
                   extra_table_cols: int = 0, name: str = "",
-                  kv_dtype: str = "bf16") -> Workload:
+                  kv_dtype: str = "bf16", q_dtype: str = "bf16") -> Workload:
     """Build a workload with explicit lengths.  Blocks are a random permutation
     of a pool of sum(ceil(S_b/BS)) + spare_blocks blocks handed out in row
     order; unused block-table slots (and ``extra_table_cols`` padding columns)
@@ -201,12 +213,17 @@ def make_workload(*, seq_lens: Sequence[int], query_lens: Sequence[int],
         v, vs = to_e4m3(v)
     elif kv_dtype != "bf16":
         raise ValueError(f"unknown kv_dtype {kv_dtype}")
+    qs = 1.0
+    if q_dtype == "fp8_e4m3":
+        q, qs = to_e4m3(q)
+    elif q_dtype != "bf16":
+        raise ValueError(f"unknown q_dtype {q_dtype}")
     return Workload(q=q, k_cache=k, v_cache=v, block_tables=tables.to(device),
                     seq_lens=torch.tensor(seq_lens, dtype=torch.int32).to(device),
                     query_lens=torch.tensor(query_lens, dtype=torch.int32).to(device),
                     windows=None if win_t is None else win_t.to(device),
                     window=int(window), scale=float(scale), name=name,
-                    k_scale=float(ks), v_scale=float(vs))
+                    k_scale=float(ks), v_scale=float(vs), q_scale=float(qs))
 
 
 def config_lengths(cfg: int):
@@ -241,7 +258,7 @@ _SHAPES = {
 
 
 def config_workload(cfg: int, device="cpu", window: Optional[int] = None,
-                    kv_dtype: str = "bf16") -> Workload:
+                    kv_dtype: str = "bf16", q_dtype: str = "bf16") -> Workload:
     """One of the five named workloads.  ``window`` overrides the scalar window
     (the tiny workload is run at window 0 and window 8); kv_dtype="fp8_e4m3"
     quantises its caches to per-tensor-scaled FP8."""
@@ -250,4 +267,4 @@ def config_workload(cfg: int, device="cpu", window: Optional[int] = None,
         w = int(window)
     return make_workload(seq_lens=s, query_lens=l, window=w, windows=ws,
                          seed=4740 + cfg, device=device, name=CONFIG_NAMES[cfg],
-                         kv_dtype=kv_dtype, **_SHAPES[cfg])
+                         kv_dtype=kv_dtype, q_dtype=q_dtype, **_SHAPES[cfg])

@@ -8,7 +8,7 @@ import numpy as np
 import torch
 
 import oracle
-from paged_kv_cache_474_b200.workloads import Workload, bf16_bits
+from paged_kv_cache_474_b200.workloads import Workload, bf16_bits, make_workload
 
 ATOL = 2e-2
 RTOL = 2e-2
@@ -20,7 +20,8 @@ def problem(wl: Workload) -> oracle.Problem:
         bf16_bits(wl.q), bf16_bits(wl.k_cache), bf16_bits(wl.v_cache),
         wl.block_tables.cpu().numpy(), wl.seq_lens.cpu().numpy(),
         wl.query_lens.cpu().numpy(), wl.scale, wl.window,
-        None if wl.windows is None else wl.windows.cpu().numpy())
+        None if wl.windows is None else wl.windows.cpu().numpy(),
+        k_scale=wl.k_scale, v_scale=wl.v_scale, q_scale=wl.q_scale)
 
 
 def subproblem(wl: Workload, rows):
@@ -54,7 +55,8 @@ def subproblem(wl: Workload, rows):
                         np.array([S[b] for b in rows], dtype=np.int32),
                         np.array([L[b] for b in rows], dtype=np.int32),
                         wl.scale, wl.window,
-                        None if W is None else np.array([W[b] for b in rows], dtype=np.int32))
+                        None if W is None else np.array([W[b] for b in rows], dtype=np.int32),
+                        k_scale=wl.k_scale, v_scale=wl.v_scale, q_scale=wl.q_scale)
     return pr, {b: j for j, b in enumerate(rows)}
 
 
@@ -105,3 +107,30 @@ def check_sampled(wl: Workload, dst, sel, what=""):
     d = dst.float().cpu().numpy()
     got = np.stack([d[qoff[b] + i, h] for b, i, h in sel])
     return assert_close(got, ref, what)
+
+
+def scaled_workload(cfg, seed=1, **kw):
+    """The named workloads' shapes at lengths the oracle finishes in seconds,
+    still spanning several stages, partitions and a ragged tail.  Extra
+    keywords (kv_dtype, q_dtype) go to make_workload."""
+    g = np.random.default_rng(seed)
+    if cfg == 2:
+        s = g.integers(100, 1500, 6).tolist()
+        return make_workload(seq_lens=s, query_lens=[1] * 6, num_q_heads=32,
+                             num_kv_heads=8, head_dim=128, block_size=16, seed=seed, **kw)
+    if cfg == 3:
+        s = g.integers(200, 2500, 7).tolist() + [300]
+        return make_workload(seq_lens=s, query_lens=[1, 1, 1, 1, 2, 3, 4, 5],
+                             num_q_heads=32, num_kv_heads=8, head_dim=128,
+                             block_size=16, window=333, seed=seed, **kw)
+    if cfg == 4:
+        return make_workload(seq_lens=[9001], query_lens=[1], num_q_heads=8,
+                             num_kv_heads=1, head_dim=128, block_size=16, seed=seed, **kw)
+    if cfg == 5:
+        s = g.integers(1100, 4200, 6).tolist()
+        l = g.integers(1, 5, 6).tolist()
+        return make_workload(seq_lens=s, query_lens=l, num_q_heads=64,
+                             num_kv_heads=8, head_dim=128, block_size=1024,
+                             windows=[700 if b % 2 == 0 else 0 for b in range(6)],
+                             seed=seed, **kw)
+    raise ValueError(cfg)

@@ -211,3 +211,44 @@ def test_plan_head_dim_256_uses_the_tensor_core_kernel():
     assert info.smem_bytes <= 227 * 1024
     rc, _ = pa.pa_plan(base_params(head_dim=256, force_variant=pa.PA_VARIANT_FMA), 16, 148, 1)
     assert rc == pa.PA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("kw", [
+    dict(kv_dtype=pa.PA_DTYPE_FP8_E4M3),                              # scales missing
+    dict(kv_dtype=pa.PA_DTYPE_FP8_E4M3, k_scale=0.5),                 # v_scale missing
+    dict(kv_dtype=pa.PA_DTYPE_FP8_E4M3, k_scale=-1.0, v_scale=1.0),
+    dict(kv_dtype=pa.PA_DTYPE_FP8_E4M3, k_scale=float("nan"), v_scale=1.0),
+    dict(kv_dtype=pa.PA_DTYPE_FP8_E4M3, k_scale=float("inf"), v_scale=1.0),
+    dict(q_dtype=pa.PA_DTYPE_FP8_E4M3),                               # q_scale missing
+    dict(q_dtype=2),
+    dict(kv_dtype=-1),
+])
+def test_fp8_operands_need_their_scales(kw):
+    # aiter PR #2914 review: FP8 tensors without their scales must be rejected
+    assert call(base_params(**kw)) == pa.PA_ERR_ARG
+    assert "scale" in pa.pa_last_error() or "dtype" in pa.pa_last_error()
+
+
+def test_fp8_scales_of_bf16_operands_are_ignored():
+    assert call(base_params(batch=0, k_scale=-5.0, q_scale=float("nan"))) == pa.PA_OK
+
+
+def test_fp8_runs_on_the_tensor_core_kernel_only():
+    kw = dict(kv_dtype=pa.PA_DTYPE_FP8_E4M3, k_scale=1.0, v_scale=1.0)
+    assert call(base_params(force_variant=pa.PA_VARIANT_FMA, **kw)) == pa.PA_ERR_UNSUPPORTED
+    kq = dict(q_dtype=pa.PA_DTYPE_FP8_E4M3, q_scale=1.0)
+    assert call(base_params(force_variant=pa.PA_VARIANT_FMA, **kq)) == pa.PA_ERR_UNSUPPORTED
+    rc, _ = pa.pa_plan(base_params(num_blocks=1 << 22, num_kv_heads=2, num_q_heads=16, **kw),
+                       1024, 148, 2)
+    assert rc == pa.PA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("d,stages", [(64, 8), (128, 4), (256, 3)])
+def test_plan_fp8_ring(d, stages):
+    info = plan(batch=8, num_q_heads=16, num_kv_heads=2, head_dim=d, num_blocks=4000,
+                max_blocks_per_seq=512, max_span_hint=8192,
+                kv_dtype=pa.PA_DTYPE_FP8_E4M3, k_scale=1.0, v_scale=1.0)
+    assert info.variant == pa.PA_VARIANT_MMA and info.stages == stages
+    # ring = stages x (K + V) x 64 tokens x head_dim bytes
+    assert info.smem_bytes >= stages * 2 * 64 * d
+    assert info.smem_bytes < stages * 2 * 64 * d + 1024 + 4096

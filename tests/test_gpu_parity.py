@@ -11,7 +11,7 @@ import torch
 
 import oracle
 from tests.parity_helpers import (assert_close, check_full, check_sampled,
-                                  problem, sample_queries, token_offsets)
+                                  problem, sample_queries, scaled_workload, token_offsets)
 
 pytestmark = pytest.mark.gpu
 
@@ -40,30 +40,7 @@ def test_tiny_workload(window, parts):
     check_full(wl, out, f"tiny w={window} parts={parts}")
 
 
-def scaled(cfg, seed=1):
-    """The named workloads' shapes at lengths the oracle finishes in seconds,
-    still spanning several stages, partitions and a ragged tail."""
-    g = np.random.default_rng(seed)
-    if cfg == 2:
-        s = g.integers(100, 1500, 6).tolist()
-        return make_workload(seq_lens=s, query_lens=[1] * 6, num_q_heads=32,
-                             num_kv_heads=8, head_dim=128, block_size=16, seed=seed)
-    if cfg == 3:
-        s = g.integers(200, 2500, 7).tolist() + [300]
-        return make_workload(seq_lens=s, query_lens=[1, 1, 1, 1, 2, 3, 4, 5],
-                             num_q_heads=32, num_kv_heads=8, head_dim=128,
-                             block_size=16, window=333, seed=seed)
-    if cfg == 4:
-        return make_workload(seq_lens=[9001], query_lens=[1], num_q_heads=8,
-                             num_kv_heads=1, head_dim=128, block_size=16, seed=seed)
-    if cfg == 5:
-        s = g.integers(1100, 4200, 6).tolist()
-        l = g.integers(1, 5, 6).tolist()
-        return make_workload(seq_lens=s, query_lens=l, num_q_heads=64,
-                             num_kv_heads=8, head_dim=128, block_size=1024,
-                             windows=[700 if b % 2 == 0 else 0 for b in range(6)],
-                             seed=seed)
-    raise ValueError(cfg)
+scaled = scaled_workload
 
 
 VARIANTS = [pa.PA_VARIANT_AUTO, pa.PA_VARIANT_FMA, pa.PA_VARIANT_MMA]

@@ -41,7 +41,7 @@ def problem_of(w, window=None, windows="keep"):
         w.block_tables.numpy(), w.seq_lens.numpy(), w.query_lens.numpy(),
         w.scale, w.window if window is None else window,
         None if ws is None else np.asarray(ws, dtype=np.int32),
-        k_scale=w.k_scale, v_scale=w.v_scale)
+        k_scale=w.k_scale, v_scale=w.v_scale, q_scale=w.q_scale)
 
 
 def cache_values(c, s):
@@ -79,7 +79,7 @@ def sdpa_reference(w, window_of_row):
         k, v = dense_kv(w, b)                      # [S, Hkv, D]
         k = k.permute(1, 0, 2).repeat_interleave(G, dim=0)  # [Hq, S, D]
         v = v.permute(1, 0, 2).repeat_interleave(G, dim=0)
-        q = w.q[qoff:qoff + L].double().permute(1, 0, 2)     # [Hq, L, D]
+        q = cache_values(w.q[qoff:qoff + L], w.q_scale).permute(1, 0, 2)  # [Hq, L, D]
         pos = torch.arange(S - L, S).unsqueeze(1)
         t = torch.arange(S).unsqueeze(0)
         win = window_of_row(b)
@@ -412,11 +412,12 @@ def test_e4m3_closed_forms(code, value):
         assert not math.copysign(1.0, oracle.e4m3_decode(np.array([0x80], np.uint8))[0]) > 0
 
 
-def fp8_mixed(window=0, windows=None, seed=13):
+def fp8_mixed(window=0, windows=None, seed=13, q_dtype="bf16", kv_dtype="fp8_e4m3"):
     return make_workload(seq_lens=[9, 23, 5, 31], query_lens=[1, 3, 5, 2],
                          num_q_heads=6, num_kv_heads=2, head_dim=16,
                          block_size=4, window=window, windows=windows,
-                         dist="normal", seed=seed, scale=0.3, kv_dtype="fp8_e4m3")
+                         dist="normal", seed=seed, scale=0.3, kv_dtype=kv_dtype,
+                         q_dtype=q_dtype)
 
 
 @pytest.mark.parametrize("window,windows", [(0, None), (5, None), (4, [3, 0, 4, 7])])
@@ -454,3 +455,22 @@ def test_fp8_split_k_invariance():
     o = oracle.decode(pr)
     for parts in (1, 2, 5):
         assert np.max(np.abs(oracle.decode(pr, parts=parts) - o)) <= 1e-13
+
+
+@pytest.mark.parametrize("q_dtype,kv_dtype", [("fp8_e4m3", "bf16"), ("fp8_e4m3", "fp8_e4m3")])
+def test_fp8_query_matches_sdpa_on_dequantised_values(q_dtype, kv_dtype):
+    w = fp8_mixed(window=5, q_dtype=q_dtype, kv_dtype=kv_dtype)
+    assert w.q_fp8 and w.q_scale > 0
+    got = oracle.decode(problem_of(w))
+    ref = sdpa_reference(w, lambda b: 5)
+    assert np.max(np.abs(got - ref)) <= 1e-12
+
+
+def test_fp8_query_scale_acts_on_the_logits():
+    w = fp8_mixed(q_dtype="fp8_e4m3")
+    pr = problem_of(w)
+    args = (pr.q, pr.k_cache, pr.v_cache, pr.block_tables, pr.seq_lens, pr.query_lens)
+    kw = dict(k_scale=w.k_scale, v_scale=w.v_scale)
+    a = oracle.decode(oracle.Problem(*args, w.scale * 1.3, q_scale=w.q_scale, **kw))
+    b = oracle.decode(oracle.Problem(*args, w.scale, q_scale=w.q_scale * 1.3, **kw))
+    assert np.max(np.abs(a - b)) <= 1e-13
