@@ -49,15 +49,17 @@ def measured_hbm_peak():
 def algorithmic_bytes(wl):
     """Bytes a call must move: K and V of every row's visible union span for
     every kv head, plus q and dst.  Union span of a row: positions
-    [max(0, S-L+1-w), S) for w > 0, [0, S) otherwise."""
+    [max(0, S-L+1-w), S) for w > 0, [0, S) otherwise.  Elements are 2 bytes
+    (bf16) or 1 (FP8 codes); dst is always bf16."""
     s, l, w = wl.host_lists()
+    kv_elem = wl.k_cache.element_size()
     kv = 0
     for S, L, W in zip(s, l, w):
         if L <= 0:
             continue
         lo = max(0, S - L + 1 - W) if W > 0 else 0
-        kv += (S - lo) * wl.num_kv_heads * 2 * wl.head_dim * 2
-    qo = 2 * wl.num_tokens * wl.num_q_heads * wl.head_dim * 2
+        kv += (S - lo) * wl.num_kv_heads * 2 * wl.head_dim * kv_elem
+    qo = wl.num_tokens * wl.num_q_heads * wl.head_dim * (wl.q.element_size() + 2)
     return kv, qo
 
 
@@ -368,15 +370,14 @@ def run_other_configs(args, local_rank):
 
     stream = torch.cuda.current_stream()
     sh = pa._stream_handle(stream)
-    res = {}
-    for cfg in (1, 2, 3, 4, 5):
-        wl = config_workload(cfg, device=device)
+
+    def measure(wl, steady_calls):
         kv, qo = algorithmic_bytes(wl)
         p = pa.params_for(wl)
         ws = pa.alloc_workspace(p, wl.block_size, device=device)
         if ws is not None:
             p.workspace, p.workspace_bytes = ws.data_ptr(), ws.numel()
-        out = torch.empty_like(wl.q)
+        out = torch.empty(wl.q.shape, dtype=torch.bfloat16, device=device)
         c = (out.data_ptr(), wl.q.data_ptr(), wl.k_cache.data_ptr(), wl.v_cache.data_ptr(),
              wl.block_tables.data_ptr(), wl.seq_lens.data_ptr(), wl.query_lens.data_ptr(),
              wl.scale, wl.window, wl.block_size)
@@ -395,41 +396,56 @@ def run_other_configs(args, local_rank):
         torch.cuda.synchronize()
         us = statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3
         gbs = (kv + qo) / (us * 1e-6) / 1e9
-        # Steady state: back-to-back calls over several copies of the KV pool
-        # (one per layer of a model, >= 4x L2 in total), so no call finds its
-        # KV in L2 and each call's launch overlaps the previous call's tail.
-        pool = wl.k_cache.numel() * wl.k_cache.element_size() * 2
-        nlay = max(1, min(64, -(-(4 * l2) // pool)))
-        layers = [(wl.k_cache, wl.v_cache)] + [(wl.k_cache.clone(), wl.v_cache.clone())
-                                               for _ in range(nlay - 1)]
-        def layer_call(i):
-            k, v = layers[i % nlay]
-            return pa.pa_decode(c[0], c[1], k.data_ptr(), v.data_ptr(), *c[4:], p, sh)
-        for i in range(nlay):
-            layer_call(i)
-        m = max(nlay, 20 if cfg == 5 else 200)
-        t0 = torch.cuda.Event(enable_timing=True)
-        t1 = torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        t0.record(stream)
-        for i in range(m):
-            layer_call(i)
-        t1.record(stream)
-        torch.cuda.synchronize()
-        us_ss = t0.elapsed_time(t1) * 1e3 / m
-        gbs_ss = (kv + qo) / (us_ss * 1e-6) / 1e9
         _, info = pa.pa_plan(p, wl.block_size)
-        res[CONFIG_NAMES[cfg]] = {"us_per_call": round(us, 2),
-                                  "kv_bytes": kv, "gbs": round(gbs, 1),
-                                  "frac_of_peak": round(gbs / peak, 4),
-                                  "l2": "flushed before each call (write then read 4x L2)",
-                                  "steady_us_per_call": round(us_ss, 2),
-                                  "steady_gbs": round(gbs_ss, 1),
-                                  "steady_frac_of_peak": round(gbs_ss / peak, 4),
-                                  "steady": f"{m} back-to-back calls over {nlay} KV pool copies",
-                                  "partitions": info.max_partitions,
-                                  "partition_tokens": info.partition_tokens}
-        del wl, ws, out, layers
+        r = {"us_per_call": round(us, 2), "kv_bytes": kv, "gbs": round(gbs, 1),
+             "frac_of_peak": round(gbs / peak, 4),
+             "l2": "flushed before each call (write then read 4x L2)",
+             "partitions": info.max_partitions, "partition_tokens": info.partition_tokens}
+        if steady_calls:
+            # Steady state: back-to-back calls over several copies of the KV
+            # pool (one per layer of a model, >= 4x L2 in total), so no call
+            # finds its KV in L2 and each call's launch overlaps the previous
+            # call's tail.
+            pool = wl.k_cache.numel() * wl.k_cache.element_size() * 2
+            nlay = max(1, min(64, -(-(4 * l2) // pool)))
+            layers = [(wl.k_cache, wl.v_cache)] + [(wl.k_cache.clone(), wl.v_cache.clone())
+                                                   for _ in range(nlay - 1)]
+
+            def layer_call(i):
+                k, v = layers[i % nlay]
+                return pa.pa_decode(c[0], c[1], k.data_ptr(), v.data_ptr(), *c[4:], p, sh)
+            for i in range(nlay):
+                layer_call(i)
+            m = max(nlay, steady_calls)
+            t0 = torch.cuda.Event(enable_timing=True)
+            t1 = torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            t0.record(stream)
+            for i in range(m):
+                layer_call(i)
+            t1.record(stream)
+            torch.cuda.synchronize()
+            us_ss = t0.elapsed_time(t1) * 1e3 / m
+            gbs_ss = (kv + qo) / (us_ss * 1e-6) / 1e9
+            r.update({"steady_us_per_call": round(us_ss, 2), "steady_gbs": round(gbs_ss, 1),
+                      "steady_frac_of_peak": round(gbs_ss / peak, 4),
+                      "steady": f"{m} back-to-back calls over {nlay} KV pool copies"})
+            del layers
+        del ws, out
+        return r
+
+    res = {}
+    for cfg in (1, 2, 3, 4, 5):
+        wl = config_workload(cfg, device=device)
+        res[CONFIG_NAMES[cfg]] = measure(wl, 20 if cfg == 5 else 200)
+        del wl
+        torch.cuda.empty_cache()
+    # The same workloads with FP8 e4m3 KV caches (per-tensor scales): half
+    # the KV bytes per token; GB/s counts the bytes actually moved.
+    for cfg in (2, 3, 4, 5):
+        wl = config_workload(cfg, device=device, kv_dtype="fp8_e4m3")
+        res[CONFIG_NAMES[cfg] + "/fp8_kv"] = measure(wl, 20 if cfg == 5 else 200)
+        del wl
         torch.cuda.empty_cache()
     # The ExecuTorch page's standalone kernel benchmark shape (B=1, H_q=16,
     # H_kv=2, D=256, one decode token) over a paged cache, per context length.
@@ -438,28 +454,9 @@ def run_other_configs(args, local_rank):
     for lk in (64, 512, 4096, 8192, 16384):
         wl = make_workload(seq_lens=[lk], query_lens=[1], num_q_heads=16, num_kv_heads=2,
                            head_dim=256, block_size=16, seed=lk, device=device)
-        kv, qo = algorithmic_bytes(wl)
-        p = pa.params_for(wl)
-        ws = pa.alloc_workspace(p, wl.block_size, device=device)
-        if ws is not None:
-            p.workspace, p.workspace_bytes = ws.data_ptr(), ws.numel()
-        out = torch.empty_like(wl.q)
-        c = (out.data_ptr(), wl.q.data_ptr(), wl.k_cache.data_ptr(), wl.v_cache.data_ptr(),
-             wl.block_tables.data_ptr(), wl.seq_lens.data_ptr(), wl.query_lens.data_ptr(),
-             wl.scale, wl.window, wl.block_size)
-        for _ in range(3):
-            pa.pa_decode(*c, p, sh)
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(20)]
-        for a, b in ev:
-            flush_l2()
-            a.record(stream)
-            pa.pa_decode(*c, p, sh)
-            b.record(stream)
-        torch.cuda.synchronize()
-        us = statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3
-        sweep[str(lk)] = {"us_per_call": round(us, 2), "gbs": round((kv + qo) / us / 1e3, 1)}
-        del wl, ws, out
+        r = measure(wl, 0)
+        sweep[str(lk)] = {"us_per_call": r["us_per_call"], "gbs": r["gbs"]}
+        del wl
     res["executorch_shape_B1_Hq16_Hkv2_D256"] = sweep
     if pa.pa_device_status(clear=True):
         raise RuntimeError("device status set during the per-config runs")

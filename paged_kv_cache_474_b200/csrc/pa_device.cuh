@@ -166,6 +166,15 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t codes16) {
   return y;
 }
 
+// Four FP8 e4m3 codes (bytes 0..3) to two f16 pairs: lo = bytes 0, 1;
+// hi = bytes 2, 3.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t codes, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(codes));
+}
+
 // bf16 pair -> f16 pair (exact for |x| in f16's normal range; larger values
 // become inf, smaller ones round to f16 subnormals).
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {

@@ -15,6 +15,7 @@
 #include <climits>
 #include <map>
 #include <mutex>
+#include <type_traits>
 #include <utility>
 
 #include <cuda.h>
@@ -432,7 +433,6 @@ template <int D, bool F8>
 struct MmaTraits {
   static constexpr int ROW_BYTES = F8 ? D : 2 * D;                  // one token of one kv head
   static constexpr int BOXW = ROW_BYTES < 128 ? ROW_BYTES : 128;    // swizzle span of a box row
-  static constexpr int HALVES = ROW_BYTES / BOXW;                   // box sub-tiles along d
   static constexpr int KV_BYTES = TS * ROW_BYTES;
   static constexpr int STAGE_BYTES = 2 * KV_BYTES;
   static constexpr int KSTEPS = D / 16;  // 16-wide reduction steps over d
@@ -733,10 +733,9 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
             ldsm_x4(Ks + cbase + box_off<T::BOXW>(lt_k, kp * 2 + ck_k, BR), r[0], r[1], r[2], r[3]);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              const uint32_t ka[4] = {e4m3x2_to_f16x2(r[2 * h] & 0xffffu),
-                                      e4m3x2_to_f16x2(r[2 * h + 1] & 0xffffu),
-                                      e4m3x2_to_f16x2(r[2 * h] >> 16),
-                                      e4m3x2_to_f16x2(r[2 * h + 1] >> 16)};
+              uint32_t ka[4];
+              e4m3x4_to_f16x2x2(r[2 * h], ka[0], ka[2]);
+              e4m3x4_to_f16x2x2(r[2 * h + 1], ka[1], ka[3]);
               const int ks = 2 * kp + h;
 #pragma unroll
               for (int n = 0; n < N8; ++n)
@@ -816,42 +815,56 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
           mk_lo = (in(t) ? 0x0000ffffu : 0u) | (in(t + 1) ? 0xffff0000u : 0u);
           mk_hi = (in(t + 8) ? 0x0000ffffu : 0u) | (in(t + 9) ? 0xffff0000u : 0u);
         }
-        if constexpr (F8) {
-          // one x4.trans = tokens 0-7 / 8-15 of chunks 2mp, 2mp+1: two M tiles;
-          // a register holds dims (2g, 2g+1) of tokens (2c, 2c+1), regrouped
-          // by dim before the conversion (the masks act on converted halves)
+        // O^T += V^T P^T; the V lanes of tokens outside [ulo, p1) are zeroed
+        // only in stages that reach past those bounds (masked = true).
+        auto pv = [&](auto masked) {
+          constexpr bool MK = decltype(masked)::value;
+          if constexpr (F8) {
+            // one x4.trans = tokens 0-7 / 8-15 of chunks 2mp, 2mp+1: two M
+            // tiles; a register holds dims (2g, 2g+1) of tokens (2c, 2c+1),
+            // regrouped by dim before the conversion (masks act on f16 halves)
 #pragma unroll
-          for (int mp = 0; mp < T::MD / 2; ++mp) {
-            uint32_t r[4];
-            ldsm_x4_t(Vs + cbase + box_off<T::BOXW>(lt_v, mp * 2 + ck_v, BR), r[0], r[1], r[2],
-                      r[3]);
+            for (int mp = 0; mp < T::MD / 2; ++mp) {
+              uint32_t r[4];
+              ldsm_x4_t(Vs + cbase + box_off<T::BOXW>(lt_v, mp * 2 + ck_v, BR), r[0], r[1], r[2],
+                        r[3]);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const uint32_t t0 = __byte_perm(r[2 * h], 0, 0x3120);
-              const uint32_t t1 = __byte_perm(r[2 * h + 1], 0, 0x3120);
-              const uint32_t va[4] = {e4m3x2_to_f16x2(t0 & 0xffffu) & mk_lo,
-                                      e4m3x2_to_f16x2(t0 >> 16) & mk_lo,
-                                      e4m3x2_to_f16x2(t1 & 0xffffu) & mk_hi,
-                                      e4m3x2_to_f16x2(t1 >> 16) & mk_hi};
+              for (int h = 0; h < 2; ++h) {
+                uint32_t va[4];
+                e4m3x4_to_f16x2x2(__byte_perm(r[2 * h], 0, 0x3120), va[0], va[1]);
+                e4m3x4_to_f16x2x2(__byte_perm(r[2 * h + 1], 0, 0x3120), va[2], va[3]);
+                if constexpr (MK) {
+                  va[0] &= mk_lo;
+                  va[1] &= mk_lo;
+                  va[2] &= mk_hi;
+                  va[3] &= mk_hi;
+                }
 #pragma unroll
-              for (int n = 0; n < N8; ++n)
-                mma_f16_16816(o[2 * mp + h][n], va, pb[n][0], pb[n][1]);
+                for (int n = 0; n < N8; ++n)
+                  mma_f16_16816(o[2 * mp + h][n], va, pb[n][0], pb[n][1]);
+              }
+            }
+          } else {
+#pragma unroll
+            for (int md = 0; md < T::MD; ++md) {
+              uint32_t va[4];
+              ldsm_x4_t(Vs + cbase + box_off<T::BOXW>(lt_v, md * 2 + ck_v, BR), va[0], va[1],
+                        va[2], va[3]);
+              if constexpr (MK) {
+                va[0] &= mk_lo;
+                va[1] &= mk_lo;
+                va[2] &= mk_hi;
+                va[3] &= mk_hi;
+              }
+#pragma unroll
+              for (int n = 0; n < N8; ++n) mma_bf16_16816(o[md][n], va, pb[n][0], pb[n][1]);
             }
           }
-        } else {
-#pragma unroll
-          for (int md = 0; md < T::MD; ++md) {
-            uint32_t va[4];
-            ldsm_x4_t(Vs + cbase + box_off<T::BOXW>(lt_v, md * 2 + ck_v, BR), va[0], va[1], va[2],
-                      va[3]);
-            va[0] &= mk_lo;
-            va[1] &= mk_lo;
-            va[2] &= mk_hi;
-            va[3] &= mk_hi;
-#pragma unroll
-            for (int n = 0; n < N8; ++n) mma_bf16_16816(o[md][n], va, pb[n][0], pb[n][1]);
-          }
-        }
+        };
+        if (boundary)
+          pv(std::true_type{});
+        else
+          pv(std::false_type{});
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars[NSTAGE + s]));
