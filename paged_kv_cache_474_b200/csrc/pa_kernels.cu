@@ -966,30 +966,55 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
 // dst = sum_p w_p O_p / sum_p w_p.  Partials are normalised, so the weights
 // carry each partition's softmax mass.
 //
-// One CTA per (row, kv head, batch row) and DSPLIT-th of head_dim.  The CTA
-// loads every lse_p once (coalesced), keeps the weights in smem, then its
-// warps sum w_p O_p: a partial's slice is DC/4 float4, so a warp reads
-// 32/(DC/4) partials per load and keeps BATCH loads in flight per lane.
-// Rows with hundreds of partials split head_dim over several CTAs so more SMs
-// pull partials from L2.  Launched with programmatic stream serialization: it
-// may be scheduled while the partition kernel drains and waits on
-// griddepcontrol before reading.
+// One CTA per (row, kv head, batch row) and DSPLIT-th of head_dim, in one
+// pass over the partials: a partial's slice is DC/4 float4, so LPP lanes
+// share a partial and a warp reads 32/LPP partials per load; each lane loads
+// lse_p with its O_p slice (BATCH partials in flight) and keeps a running
+// (max, sum, weighted sum), merged across the lanes of a slice and then
+// across warps with the same rescale.  Only the lengths are read before the
+// partials, so a row costs two dependent trips to L2.  Rows with hundreds of
+// partials split head_dim over several CTAs so more SMs pull partials from
+// L2.  Launched with programmatic stream serialization: it may be scheduled
+// while the partition kernel drains and waits on griddepcontrol before
+// reading.
 // ---------------------------------------------------------------------------
+struct LseAcc {
+  float m, z;
+  float4 o;
+};
+
+// (m, z, o) += (m2, z2, o2) with the larger maximum kept; -inf maxima weigh 0.
+__device__ __forceinline__ void lse_merge(LseAcc& x, float m2, float z2, float4 o2) {
+  const float mn = fmaxf(x.m, m2);
+  const float f1 = mn == kNegInf ? 0.f : ex2(x.m - mn);
+  const float f2 = mn == kNegInf ? 0.f : ex2(m2 - mn);
+  x.z = x.z * f1 + z2 * f2;
+  x.o.x = x.o.x * f1 + o2.x * f2;
+  x.o.y = x.o.y * f1 + o2.y * f2;
+  x.o.z = x.o.z * f1 + o2.z * f2;
+  x.o.w = x.o.w * f1 + o2.w * f2;
+  x.m = mn;
+}
+
 template <int D, int DSPLIT>
 __global__ void __launch_bounds__(512) pa_reduce_kernel(const __grid_constant__ DecodeArgs a) {
   constexpr int DC = D / DSPLIT;  // dims per CTA
   constexpr int LPP = DC / 4;     // lanes per partial slice (one float4 each)
   constexpr int PPW = 32 / LPP;   // partials per warp load
-  constexpr int BATCH = 8;        // loads in flight per lane
-  extern __shared__ float s_w[];  // [max_parts] weights
-  __shared__ float s_red[16];
-  __shared__ float4 s_acc[16][LPP];
-  __shared__ float s_M, s_Z;
+  constexpr int BATCH = 8;        // partials in flight per lane
+  __shared__ float s_m[16], s_z[16];
+  __shared__ float4 s_o[16][LPP];
   __shared__ int s_qoff;
 
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int rr = blockIdx.x / DSPLIT, ch = blockIdx.x - (blockIdx.x / DSPLIT) * DSPLIT;
   const int kvh = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nw = blockDim.x >> 5;
+  if (warp == 0) {
+    const int q0 = row_token_offset(a.query_lens, b, lane);
+    if (lane == 0) s_qoff = q0;
+  }
   const int S = a.seq_lens[b];
   const int L = a.query_lens[b];
   const int w = a.windows ? a.windows[b] : a.window;
@@ -1000,97 +1025,56 @@ __global__ void __launch_bounds__(512) pa_reduce_kernel(const __grid_constant__ 
   const int nparts = (S - A + a.part_tokens - 1) / a.part_tokens;
   if (nparts <= 1 || nparts > a.max_parts) return;
 
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nw = blockDim.x >> 5;
-  if (warp == 0) {
-    const int q0 = row_token_offset(a.query_lens, b, lane);
-    if (lane == 0) s_qoff = q0;
-  }
+  const int sub = lane / LPP, c4 = lane - (lane / LPP) * LPP;
   const size_t ubase = (size_t)(b * a.num_kv_heads + kvh) * a.max_parts;
   const float* lse = a.ws_lse + ubase * a.max_rows + rr;
-
-  float m = kNegInf;
-  for (int p = tid; p < nparts; p += blockDim.x) {
-    const float v = lse[(size_t)p * a.max_rows];
-    s_w[p] = v;
-    m = fmaxf(m, v);
-  }
-#pragma unroll
-  for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
-  if (lane == 0) s_red[warp] = m;
-  __syncthreads();
-  if (tid == 0) {
-    float x = s_red[0];
-    for (int i = 1; i < nw; ++i) x = fmaxf(x, s_red[i]);
-    s_M = x;
-  }
-  __syncthreads();
-  const float M = s_M;
-  float z = 0.f;
-  for (int p = tid; p < nparts; p += blockDim.x) {
-    const float wt = ex2(s_w[p] - M);  // an empty partition (-inf) weighs 0
-    s_w[p] = wt;
-    z += wt;
-  }
-#pragma unroll
-  for (int o = 16; o; o >>= 1) z += __shfl_xor_sync(FULL, z, o);
-  __syncthreads();
-  if (lane == 0) s_red[warp] = z;
-  __syncthreads();
-  if (tid == 0) {
-    float x = 0.f;
-    for (int i = 0; i < nw; ++i) x += s_red[i];
-    s_Z = x;
-  }
-
-  const int sub = lane / LPP, c4 = lane - (lane / LPP) * LPP;
   const float4* ob =
       reinterpret_cast<const float4*>(a.ws_o + (ubase * a.max_rows + rr) * D + ch * DC) + c4;
   const size_t pst4 = (size_t)a.max_rows * D / 4;  // float4 stride between partials
   const int step = nw * PPW;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  LseAcc acc{kNegInf, 0.f, make_float4(0.f, 0.f, 0.f, 0.f)};
   for (int p0 = warp * PPW + sub; p0 < nparts; p0 += BATCH * step) {
+    float l[BATCH];
     float4 o[BATCH];
 #pragma unroll
     for (int u = 0; u < BATCH; ++u) {
       const int p = p0 + u * step;
+      l[u] = p < nparts ? lse[(size_t)p * a.max_rows] : kNegInf;
       o[u] = p < nparts ? ob[(size_t)p * pst4] : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
-    for (int u = 0; u < BATCH; ++u) {
-      const int p = p0 + u * step;
-      const float wt = p < nparts ? s_w[p] : 0.f;
-      acc.x += wt * o[u].x;
-      acc.y += wt * o[u].y;
-      acc.z += wt * o[u].z;
-      acc.w += wt * o[u].w;
-    }
+    for (int u = 0; u < BATCH; ++u) lse_merge(acc, l[u], 1.f, o[u]);
   }
+  // lanes holding the same dims (c4) in other slices of the warp
 #pragma unroll
   for (int off = LPP; off < 32; off <<= 1) {
-    acc.x += __shfl_xor_sync(FULL, acc.x, off);
-    acc.y += __shfl_xor_sync(FULL, acc.y, off);
-    acc.z += __shfl_xor_sync(FULL, acc.z, off);
-    acc.w += __shfl_xor_sync(FULL, acc.w, off);
+    const float m2 = __shfl_xor_sync(FULL, acc.m, off);
+    const float z2 = __shfl_xor_sync(FULL, acc.z, off);
+    float4 o2;
+    o2.x = __shfl_xor_sync(FULL, acc.o.x, off);
+    o2.y = __shfl_xor_sync(FULL, acc.o.y, off);
+    o2.z = __shfl_xor_sync(FULL, acc.o.z, off);
+    o2.w = __shfl_xor_sync(FULL, acc.o.w, off);
+    lse_merge(acc, m2, z2, o2);
   }
-  if (sub == 0) s_acc[warp][c4] = acc;
+  if (sub == 0) {
+    s_o[warp][c4] = acc.o;
+    if (c4 == 0) {
+      s_m[warp] = acc.m;
+      s_z[warp] = acc.z;
+    }
+  }
   __syncthreads();
   if (warp == 0 && lane < LPP) {
-    float4 out = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int i = 0; i < nw; ++i) {
-      const float4 v = s_acc[i][lane];
-      out.x += v.x;
-      out.y += v.y;
-      out.z += v.z;
-      out.w += v.w;
-    }
-    const float inv = 1.f / s_Z;
+    LseAcc t{kNegInf, 0.f, make_float4(0.f, 0.f, 0.f, 0.f)};
+    for (int i = 0; i < nw; ++i) lse_merge(t, s_m[i], s_z[i], s_o[i][lane]);
+    const float inv = t.z > 0.f ? 1.f / t.z : 0.f;
     const int i = rr / a.group, j = rr - (rr / a.group) * a.group;
     __nv_bfloat16* dp = a.dst +
                         ((size_t)(s_qoff + i) * a.num_q_heads + (size_t)kvh * a.group + j) * D +
                         ch * DC + lane * 4;
-    *reinterpret_cast<__nv_bfloat162*>(dp) = __floats2bfloat162_rn(out.x * inv, out.y * inv);
-    *reinterpret_cast<__nv_bfloat162*>(dp + 2) = __floats2bfloat162_rn(out.z * inv, out.w * inv);
+    *reinterpret_cast<__nv_bfloat162*>(dp) = __floats2bfloat162_rn(t.o.x * inv, t.o.y * inv);
+    *reinterpret_cast<__nv_bfloat162*>(dp + 2) = __floats2bfloat162_rn(t.o.z * inv, t.o.w * inv);
   }
 }
 
@@ -1325,7 +1309,7 @@ cudaError_t launch_reduce_t(const DecodeArgs& a, cudaStream_t stream) {
   // warps so that each lane has about one batch of eight loads, 1 to 16
   const int nw = max(1, min(16, (a.max_parts + PPW * 8 - 1) / (PPW * 8)));
   cfg.blockDim = dim3(32 * nw);
-  cfg.dynamicSmemBytes = (size_t)a.max_parts * sizeof(float);
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -1333,11 +1317,6 @@ cudaError_t launch_reduce_t(const DecodeArgs& a, cudaStream_t stream) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   auto kern = pa_reduce_kernel<D, DSPLIT>;
-  if (cfg.dynamicSmemBytes > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)cfg.dynamicSmemBytes);
-    if (e != cudaSuccess) return e;
-  }
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
