@@ -83,6 +83,8 @@ extern "C" {
 #define PA_VARIANT_AUTO 0
 #define PA_VARIANT_FMA 1      /* CUDA-core FMA scores and PV (group x queryLen <= 4 rows) */
 #define PA_VARIANT_MMA 2      /* tensor-core m16n8k16 tiles with TMA-swizzled staging (dense rows) */
+#define PA_VARIANT_TC 3       /* tcgen05 MMAs on FP8 codes in shared memory, accumulators in tensor
+                                 memory (FP8 caches, head_dim 128; 8 rows per CTA) */
 
 typedef struct pa_params {
     int batch;               /* rows */

@@ -32,6 +32,7 @@ PA_DEV_HINT = 8
 PA_VARIANT_AUTO = 0
 PA_VARIANT_FMA = 1
 PA_VARIANT_MMA = 2
+PA_VARIANT_TC = 3
 
 PA_DTYPE_BF16 = 0
 PA_DTYPE_FP8_E4M3 = 1

@@ -106,7 +106,7 @@ int check_params(const pa_params* p, int bs) {
     return fail(PA_ERR_ARG, "hints must be >= 0");
   if (p->force_partitions < 0) return fail(PA_ERR_ARG, "force_partitions must be >= 0");
   if (p->force_variant != PA_VARIANT_AUTO && p->force_variant != PA_VARIANT_FMA &&
-      p->force_variant != PA_VARIANT_MMA)
+      p->force_variant != PA_VARIANT_MMA && p->force_variant != PA_VARIANT_TC)
     return fail(PA_ERR_ARG, "unknown force_variant %d", p->force_variant);
   // FP8 operands need their scales (aiter PR #2914 review: validate that
   // query_scale / key_scale / value_scale are present for FP8 tensors).
@@ -128,18 +128,21 @@ bool any_fp8(const pa_params* p) {
 
 // Resident CTAs per SM of a kernel instance, queried once per device.
 int cached_occupancy(bool mma, const pa::KernelShape& k, size_t smem) {
+  // (k.tc selects the tensor-memory kernel)
   static std::mutex mu;
   static std::map<std::vector<long long>, int> cache;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
   const std::vector<long long> key = {dev, mma, k.head_dim, k.consumer_warps, k.stages, k.n8,
-                                      k.kv_fp8, (long long)smem};
+                                      k.kv_fp8, k.tc, (long long)smem};
   {
     std::lock_guard<std::mutex> lock(mu);
     auto it = cache.find(key);
     if (it != cache.end()) return it->second;
   }
-  const int n = mma ? pa::occupancy_partition_mma(k, smem) : pa::occupancy_partition_fma(k, smem);
+  const int n = k.tc ? pa::occupancy_partition_tc(k, smem)
+                : mma  ? pa::occupancy_partition_mma(k, smem)
+                       : pa::occupancy_partition_fma(k, smem);
   if (n > 0) {
     std::lock_guard<std::mutex> lock(mu);
     cache[key] = n;
@@ -171,40 +174,61 @@ int make_plan(const pa_params* p, int bs, int span, int qlen, int num_sms, int c
   // m16n8k16 replaces ~40 FMA-path instructions per token.  The FMA kernel
   // stays for pools whose row count exceeds the TMA map's 32-bit
   // coordinates, and on request.
+  //
+  // The tensor-memory kernel (FP8 caches, head_dim 128) runs on request: it
+  // feeds the e4m3 codes to tcgen05 straight from shared memory, but its
+  // softmax warps (one token per thread, eight per SM) are latency-bound and
+  // it trails the mma.sync kernel on the named workloads (GQA decode FP8:
+  // 97 vs 75 us).
   const bool rows_fit_tma =
       (long long)p->num_blocks * p->num_kv_heads * bs <= (long long)INT32_MAX;
+  const bool kv8 = p->kv_dtype == PA_DTYPE_FP8_E4M3;
+  const bool tc_shape = kv8 && p->head_dim == 128 && rows_fit_tma;
   int variant = p->force_variant;
   if (variant == PA_VARIANT_AUTO) variant = rows_fit_tma ? PA_VARIANT_MMA : PA_VARIANT_FMA;
   if (variant == PA_VARIANT_MMA && !rows_fit_tma)
     return fail(PA_ERR_UNSUPPORTED, "KV pool rows exceed the tensor map's 32-bit coordinates");
+  if (variant == PA_VARIANT_TC && !tc_shape)
+    return fail(PA_ERR_UNSUPPORTED,
+                "the tensor-memory variant needs FP8 caches, head_dim 128 and a pool within the "
+                "tensor map's 32-bit rows");
+  const bool tc = variant == PA_VARIANT_TC;
   if (variant == PA_VARIANT_FMA && p->head_dim == 256)
     return fail(PA_ERR_UNSUPPORTED, "head_dim 256 runs on the tensor-core kernel only");
   if (variant == PA_VARIANT_FMA && any_fp8(p))
     return fail(PA_ERR_UNSUPPORTED, "FP8 operands run on the tensor-core kernel only");
-  const bool mma = variant == PA_VARIANT_MMA;
-  const bool kv8 = p->kv_dtype == PA_DTYPE_FP8_E4M3;
+  const bool mma = variant == PA_VARIANT_MMA || tc;  // TMA-staged kernels
   const int ncw = mma ? 4 : (rmax <= 16 ? 4 : 8);
   // tensor-core warps cover 8 rows (one n-tile) when the unit has <= 8 rows,
   // else 16 (head_dim 256: always 8, its accumulators are twice as wide); a
   // CTA covers up to 4 such tiles.
-  const int n8 = (mma && rmax > 8 && p->head_dim <= 128) ? 2 : 1;
+  const int n8 = (mma && !tc && rmax > 8 && p->head_dim <= 128) ? 2 : 1;
   pl.shape.n8 = n8;
-  const int slab_rows = mma ? 8 * n8 * ncw : 4 * ncw;
+  pl.shape.tc = tc;
+  // the tensor-memory kernel covers 8 rows per CTA (its MMA's N is 16)
+  const int slab_rows = tc ? 8 : mma ? 8 * n8 * ncw : 4 * ncw;
   const int nslab = (int)cdiv(rmax, slab_rows);
   pl.shape.head_dim = p->head_dim;
   pl.shape.consumer_warps = ncw;
   pl.shape.kv_fp8 = kv8;
   // bf16: 16, 32 or 64 KB per stage; FP8: 8, 16 or 32 KB per stage
-  if (!kv8)
+  if (tc)
+    pl.shape.stages = 3;  // 32 KB (128 tokens) per stage
+  else if (!kv8)
     pl.shape.stages = p->head_dim == 64 ? 4 : 3;
   else
     pl.shape.stages = p->head_dim == 64 ? 8 : p->head_dim == 128 ? 4 : 3;
 
-  // Partition-size cap: the CTA caches its slice of the block table in smem.
-  const int cap = std::max(TS, ((pa::kMaxTableCache - 2) * bs) / TS * TS);
+  // Partitions are whole stages: 64 tokens, 128 for the tensor-memory kernel.
+  const int unit = tc ? 2 * TS : TS;
+  // Partition-size cap: the CTA caches its slice of the block table in smem
+  // (the tensor-memory kernel keeps it to 4096 tokens so two CTAs fit an SM).
+  int cap = std::max(unit, ((pa::kMaxTableCache - 2) * bs) / unit * unit);
+  if (tc) cap = std::min(cap, 4096);
   auto smem_for = [&](int ptok) {
-    return mma ? pa::mma_smem_bytes(p->head_dim, kv8 ? 1 : 2, pl.shape.stages, ptok, bs)
-               : pa::fma_smem_bytes(p->head_dim, pl.shape.stages, ptok, bs);
+    return tc    ? pa::tc_smem_bytes(pl.shape.stages, ptok, bs)
+           : mma ? pa::mma_smem_bytes(p->head_dim, kv8 ? 1 : 2, pl.shape.stages, ptok, bs)
+                 : pa::fma_smem_bytes(p->head_dim, pl.shape.stages, ptok, bs);
   };
   if (num_sms <= 0) {
     int rc = current_sms(&num_sms);
@@ -220,12 +244,12 @@ int make_plan(const pa_params* p, int bs, int span, int qlen, int num_sms, int c
 
   long long ptok;
   if (p->force_partitions > 0) {
-    ptok = cdiv(cdiv(span, p->force_partitions), TS) * TS;
+    ptok = cdiv(cdiv(span, p->force_partitions), unit) * unit;
   } else {
     if (units * 4 <= slots) {
       // few units: one balanced wave over every resident-CTA slot
       const long long want = std::max<long long>(1, cdiv(slots, std::max<long long>(units, 1)));
-      ptok = std::max<long long>(cdiv(cdiv(span, want), TS) * TS, kMinPartTokens);
+      ptok = std::max<long long>(cdiv(cdiv(span, want), unit) * unit, kMinPartTokens);
     } else {
       // many units: about four waves, but partitions of 2048..4096 tokens,
       // long enough to amortise a CTA's start-up and short enough that
@@ -237,12 +261,12 @@ int make_plan(const pa_params* p, int bs, int span, int qlen, int num_sms, int c
       // a multiple of the target does not end in a sliver partition
       const long long aligned_span = (long long)span + TS - 1;
       const long long np = std::max<long long>(1, (aligned_span + target / 2) / target);
-      ptok = cdiv(cdiv(aligned_span, np), TS) * TS;
+      ptok = cdiv(cdiv(aligned_span, np), unit) * unit;
     }
   }
-  ptok = std::min<long long>(std::max<long long>(ptok, TS), cap);
-  // The reduce keeps one weight per partition in smem: at most 16384.
-  ptok = std::max<long long>(ptok, cdiv(cdiv((long long)span + TS - 1, 16384), TS) * TS);
+  ptok = std::min<long long>(std::max<long long>(ptok, unit), cap);
+  // At most 16384 partitions per row.
+  ptok = std::max<long long>(ptok, cdiv(cdiv((long long)span + TS - 1, 16384), unit) * unit);
   const long long max_parts = cdiv((long long)span + TS - 1, ptok);
   if (max_parts > 16384) return fail(PA_ERR_UNSUPPORTED, "too many partitions");
 
@@ -258,7 +282,7 @@ int make_plan(const pa_params* p, int bs, int span, int qlen, int num_sms, int c
   in.grid_x = (int)max_parts;
   in.grid_y = p->num_kv_heads * nslab;
   in.grid_z = p->batch;
-  in.block_threads = 32 * (ncw + 1);
+  in.block_threads = tc ? 192 : 32 * (ncw + 1);
   in.smem_bytes = smem_for((int)ptok);
   in.num_sms = num_sms;
   in.ctas_per_sm = ctas_per_sm;
@@ -442,7 +466,7 @@ int decode_impl(void* dst, const void* q, const void* kCache, const void* vCache
   }
   cudaError_t e = ev0 ? cudaEventRecord(ev0, stream) : cudaSuccess;
   if (e == cudaSuccess) {
-    if (in.variant == PA_VARIANT_MMA) {
+    if (in.variant == PA_VARIANT_MMA || in.variant == PA_VARIANT_TC) {
       CUtensorMap tk, tv;
       const long long rows = (long long)p->num_blocks * p->num_kv_heads * bs;
       const int br = std::min(bs, TS);
@@ -450,7 +474,9 @@ int decode_impl(void* dst, const void* q, const void* kCache, const void* vCache
       rc = kv_tensor_map(&tk, kCache, rows, p->head_dim, eb, br);
       if (!rc) rc = kv_tensor_map(&tv, vCache, rows, p->head_dim, eb, br);
       if (rc) return rc;
-      e = pa::launch_partition_mma(a, pl.shape, tk, tv, grid, in.smem_bytes, stream);
+      e = in.variant == PA_VARIANT_TC
+              ? pa::launch_partition_tc(a, pl.shape, tk, tv, grid, in.smem_bytes, stream)
+              : pa::launch_partition_mma(a, pl.shape, tk, tv, grid, in.smem_bytes, stream);
     } else {
       e = pa::launch_partition_fma(a, pl.shape, grid, in.smem_bytes, stream);
     }

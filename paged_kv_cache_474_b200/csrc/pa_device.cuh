@@ -175,6 +175,14 @@ __device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t codes, uint32_t& lo, 
       : "r"(codes));
 }
 
+// Two floats to two e4m3 codes (round to nearest even, saturating at
+// +-448); lo goes to the low byte.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+  unsigned short y;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(y) : "f"(hi), "f"(lo));
+  return y;
+}
+
 // bf16 pair -> f16 pair (exact for |x| in f16's normal range; larger values
 // become inf, smaller ones round to f16 subnormals).
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {

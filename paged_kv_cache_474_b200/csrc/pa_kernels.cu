@@ -12,6 +12,7 @@
 // through a shared-memory ring with the TMA engine's bulk copies
 // (cp.async.bulk + mbarrier transaction counts); compute warps read each
 // staged K/V row once for every query row of the GQA group.
+#include <algorithm>
 #include <climits>
 #include <map>
 #include <mutex>
@@ -1225,7 +1226,75 @@ int occupancy_mma_t(size_t smem) {
   return n;
 }
 
+
+#include "pa_tc.cuh"
+
+template <int NS, int RT>
+cudaError_t launch_tc_t(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
+                        dim3 grid, size_t smem, cudaStream_t stream) {
+  auto kern = pa_partition_tc_kernel<NS, RT>;
+  cudaError_t e = ensure_smem_attrs(reinterpret_cast<const void*>(kern), smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a, tk, tv);
+}
+
+// Resident CTAs per SM from the kernel's own limits.  (The runtime's
+// occupancy query answers 1 for this kernel at any shared-memory size, while
+// two CTAs per SM are observed resident on B200, as shared memory, registers
+// and tensor memory allow.)
+template <int NS, int RT>
+int occupancy_tc_t(size_t smem) {
+  auto kern = pa_partition_tc_kernel<NS, RT>;
+  if (ensure_smem_attrs(reinterpret_cast<const void*>(kern), smem) != cudaSuccess) return 0;
+  cudaFuncAttributes fa;
+  int dev = 0, sm_smem = 0, sm_regs = 0, reserved = 0;
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sm_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) !=
+          cudaSuccess ||
+      cudaDeviceGetAttribute(&sm_regs, cudaDevAttrMaxRegistersPerMultiprocessor, dev) !=
+          cudaSuccess ||
+      cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, dev) !=
+          cudaSuccess)
+    return 0;
+  const long long per_cta_smem = (long long)smem + (long long)fa.sharedSizeBytes + reserved;
+  const int regs = ((fa.numRegs + 7) / 8) * 8;  // allocated per thread in units of 8
+  int n = (int)(sm_smem / per_cta_smem);
+  n = std::min(n, sm_regs / (regs * 192));
+  n = std::min(n, 512 / kTcTmemCols);  // tensor-memory columns per SM
+  return std::max(n, 0);
+}
+
 }  // namespace
+
+size_t tc_smem_bytes(int stages, int part_tokens, int block_size) {
+  const size_t nbt = (size_t)part_tokens / block_size + 2;
+  return 1024 + (size_t)stages * TcLayout::STAGE_BYTES + 2 * TcLayout::QB_BYTES +
+         4 * TcLayout::PB_BYTES + (2 * (size_t)stages + 9) * sizeof(uint64_t) +
+         (2 * 4 + 4 + 4 + 1) * kTcN * sizeof(float) + nbt * sizeof(int);
+}
+
+cudaError_t launch_partition_tc(const DecodeArgs& a, const KernelShape& k, const CUtensorMap& tk,
+                                const CUtensorMap& tv, dim3 grid, size_t smem,
+                                cudaStream_t stream) {
+  if (k.head_dim == 128 && k.stages == 3 && k.n8 == 1 && k.kv_fp8)
+    return launch_tc_t<3, 8>(a, tk, tv, grid, smem, stream);
+  return cudaErrorInvalidValue;
+}
+
+int occupancy_partition_tc(const KernelShape& k, size_t smem) {
+  if (k.head_dim == 128 && k.stages == 3 && k.n8 == 1 && k.kv_fp8) return occupancy_tc_t<3, 8>(smem);
+  return 0;
+}
 
 size_t mma_smem_bytes(int head_dim, int elem_bytes, int stages, int part_tokens, int block_size) {
   const size_t ring = (size_t)stages * 2 * TS * head_dim * elem_bytes;

@@ -46,6 +46,7 @@ struct KernelShape {
   int stages;
   int n8;  // tensor-core variant: 8-row n-tiles per compute warp (1 or 2)
   int kv_fp8;  // tensor-core variant: FP8 e4m3 K/V caches
+  int tc;      // tensor-memory (tcgen05) variant
 };
 
 // Dynamic shared memory of the FMA partition kernel.
@@ -70,6 +71,18 @@ cudaError_t launch_partition_mma(const DecodeArgs& a, const KernelShape& k, cons
                                  cudaStream_t stream);
 
 int occupancy_partition_mma(const KernelShape& k, size_t smem);
+
+// Dynamic shared memory of the tensor-memory (tcgen05) partition kernel
+// (FP8 caches, head_dim 128, 128-token stages).
+size_t tc_smem_bytes(int stages, int part_tokens, int block_size);
+
+// Launches the tcgen05 partition kernel (192 threads); tk / tv as for the
+// tensor-core kernel with FP8 caches.
+cudaError_t launch_partition_tc(const DecodeArgs& a, const KernelShape& k, const CUtensorMap& tk,
+                                const CUtensorMap& tv, dim3 grid, size_t smem,
+                                cudaStream_t stream);
+
+int occupancy_partition_tc(const KernelShape& k, size_t smem);
 
 // Launches the log-sum-exp reduce over (rows, kv heads, batch).
 cudaError_t launch_reduce(const DecodeArgs& a, cudaStream_t stream);

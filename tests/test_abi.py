@@ -60,6 +60,7 @@ def call(p, bs=16, window=0, scale=0.125, ptrs=16):
     (dict(max_span_hint=-3), pa.PA_ERR_ARG),
     (dict(force_partitions=-1), pa.PA_ERR_ARG),
     (dict(force_variant=7), pa.PA_ERR_ARG),
+    (dict(force_variant=4), pa.PA_ERR_ARG),
 ])
 def test_invalid_params_are_rejected_on_the_host(kw, code):
     assert call(base_params(**kw)) == code
@@ -246,9 +247,32 @@ def test_fp8_runs_on_the_tensor_core_kernel_only():
 @pytest.mark.parametrize("d,stages", [(64, 8), (128, 4), (256, 3)])
 def test_plan_fp8_ring(d, stages):
     info = plan(batch=8, num_q_heads=16, num_kv_heads=2, head_dim=d, num_blocks=4000,
-                max_blocks_per_seq=512, max_span_hint=8192,
+                max_blocks_per_seq=512, max_span_hint=8192, force_variant=pa.PA_VARIANT_MMA,
                 kv_dtype=pa.PA_DTYPE_FP8_E4M3, k_scale=1.0, v_scale=1.0)
     assert info.variant == pa.PA_VARIANT_MMA and info.stages == stages
     # ring = stages x (K + V) x 64 tokens x head_dim bytes
     assert info.smem_bytes >= stages * 2 * 64 * d
     assert info.smem_bytes < stages * 2 * 64 * d + 1024 + 4096
+
+
+def test_plan_tensor_memory_variant_on_request():
+    fp8 = dict(kv_dtype=pa.PA_DTYPE_FP8_E4M3, k_scale=1.0, v_scale=1.0)
+    gqa = dict(batch=32, num_q_heads=32, num_kv_heads=8, head_dim=128, num_blocks=20000,
+               max_blocks_per_seq=512, max_span_hint=8192)
+    assert plan(**gqa, **fp8).variant == pa.PA_VARIANT_MMA   # not chosen by itself
+    info = plan(force_variant=pa.PA_VARIANT_TC, **gqa, **fp8)
+    assert info.variant == pa.PA_VARIANT_TC and info.block_threads == 192
+    assert info.slab_rows == 8 and info.stages == 3
+    assert info.partition_tokens % 128 == 0
+    # more rows run as 8-row slabs; bf16 caches and other head dims are refused
+    forced = plan(force_variant=pa.PA_VARIANT_TC, **dict(gqa, max_query_len_hint=3), **fp8)
+    assert forced.variant == pa.PA_VARIANT_TC and forced.grid_y == 8 * 2
+    rc, _ = pa.pa_plan(base_params(force_variant=pa.PA_VARIANT_TC, **gqa), 16, 148, 2)
+    assert rc == pa.PA_ERR_UNSUPPORTED
+    rc, _ = pa.pa_plan(base_params(force_variant=pa.PA_VARIANT_TC, **dict(gqa, head_dim=64),
+                                   **fp8), 16, 148, 2)
+    assert rc == pa.PA_ERR_UNSUPPORTED
+    long_row = plan(batch=1, num_q_heads=8, num_kv_heads=1, head_dim=128, num_blocks=8193,
+                    max_blocks_per_seq=8192, max_span_hint=131072,
+                    force_variant=pa.PA_VARIANT_TC, **fp8)
+    assert long_row.variant == pa.PA_VARIANT_TC and long_row.partition_tokens % 128 == 0

@@ -198,3 +198,108 @@ def test_missing_scale_is_rejected_before_launch():
                       wl.block_size, p, pa._stream_handle())
     assert rc == pa.PA_ERR_ARG and "v_scale" in pa.pa_last_error()
     assert not out.any()
+
+
+# ------------------------------------------- tensor-memory (tcgen05) kernel
+TC = pa.PA_VARIANT_TC
+
+
+def _variant_of(wl, **kw):
+    _, info = pa.pa_plan(pa.params_for(dev(wl), **kw), wl.block_size)
+    return info.variant
+
+
+@pytest.mark.parametrize("variant", [pa.PA_VARIANT_MMA, TC])
+@pytest.mark.parametrize("cfg", [2, 3, 4, 5])
+@pytest.mark.parametrize("parts", [0, 1, 5])
+def test_tensor_memory_kernel_on_the_named_shapes(cfg, parts, variant):
+    # the forced tensor-memory kernel runs units of more than 8 rows as slabs
+    wl = scaled_workload(cfg, kv_dtype=FP8, seed=3)
+    assert _variant_of(wl, force_variant=variant) == variant
+    out = pa.decode(dev(wl), force_partitions=parts, force_variant=variant)
+    check_full(wl, out, f"cfg{cfg} parts={parts} variant={variant}")
+
+
+def test_tensor_memory_kernel_runs_on_request_only():
+    assert _variant_of(scaled_workload(2, kv_dtype=FP8)) == pa.PA_VARIANT_MMA
+    assert _variant_of(scaled_workload(2, kv_dtype=FP8), force_variant=TC) == TC
+
+
+@pytest.mark.parametrize("block_size", [16, 32, 64, 256, 1024])
+@pytest.mark.parametrize("q_dtype", ["bf16", FP8])
+def test_tensor_memory_kernel_block_sizes_and_queries(block_size, q_dtype):
+    wl = make_workload(seq_lens=[1, 17, 64, 65, 127, 128, 129, 1500, 2049],
+                       query_lens=[1, 1, 2, 1, 1, 1, 3, 4, 1], num_q_heads=8, num_kv_heads=4,
+                       head_dim=128, block_size=block_size, window=0, seed=block_size,
+                       kv_dtype=FP8, q_dtype=q_dtype)
+    out = pa.decode(dev(wl), force_variant=TC)
+    check_full(wl, out, f"tc BS={block_size} q={q_dtype}")
+
+
+@pytest.mark.parametrize("group,qlen", [(1, 1), (2, 3), (4, 2), (8, 1), (8, 2), (16, 1)])
+def test_tensor_memory_kernel_rows_and_slabs(group, qlen):
+    wl = make_workload(seq_lens=[700, 64, 1999], query_lens=[qlen, min(qlen, 2), qlen],
+                       num_q_heads=2 * group, num_kv_heads=2, head_dim=128, block_size=16,
+                       windows=[100, 0, 33], seed=group * 10 + qlen, kv_dtype=FP8)
+    out = pa.decode(dev(wl), force_variant=TC)
+    check_full(wl, out, f"tc group={group} qlen={qlen}")
+
+
+@pytest.mark.parametrize("parts", [1, 2, 3, 7, 64, 200])
+def test_tensor_memory_kernel_split_k(parts):
+    wl = make_workload(seq_lens=[5000, 3333, 77], query_lens=[1, 3, 2], num_q_heads=8,
+                       num_kv_heads=4, head_dim=128, block_size=16, window=0, seed=7,
+                       kv_dtype=FP8)
+    out = pa.decode(dev(wl), force_partitions=parts, force_variant=TC)
+    check_full(wl, out, f"tc parts={parts}")
+
+
+def test_tensor_memory_kernel_never_reads_outside_spans():
+    wl = make_workload(seq_lens=[1000, 333, 77, 50], query_lens=[3, 1, 2, 1], num_q_heads=8,
+                       num_kv_heads=4, head_dim=128, block_size=16,
+                       windows=[50, 0, 20, 0], seed=19, spare_blocks=2, extra_table_cols=3,
+                       kv_dtype=FP8)
+    ref = oracle.decode(problem(wl))
+    W = wl.windows.tolist()
+    for b, (S, L) in enumerate(zip(wl.seq_lens.tolist(), wl.query_lens.tolist())):
+        nb = (S + 15) // 16
+        last = int(wl.block_tables[b, nb - 1])
+        wl.k_cache[last, :, S - (nb - 1) * 16:] = NAN_CODE
+        wl.v_cache[last, :, S - (nb - 1) * 16:] = NAN_CODE
+        first = max(0, S - L + 1 - W[b]) if W[b] > 0 else 0
+        for t in range(first):
+            blk = int(wl.block_tables[b, t // 16])
+            wl.k_cache[blk, :, t % 16] = NAN_CODE
+            wl.v_cache[blk, :, t % 16] = NAN_CODE
+        wl.block_tables[b, nb:] = 10 ** 6
+    used = set(wl.block_tables[wl.block_tables < wl.num_blocks].tolist())
+    for blk in range(wl.num_blocks):
+        if blk not in used:
+            wl.k_cache[blk] = NAN_CODE
+            wl.v_cache[blk] = NAN_CODE
+    out = pa.decode(dev(wl), force_variant=TC)
+    assert_close(out.float().cpu().numpy(), ref, "tc NaN codes outside spans")
+
+
+def test_tensor_memory_kernel_large_and_tiny_queries():
+    # a bf16 q row is split into two e4m3 terms after a power-of-two scale:
+    # rows of very different magnitudes must all come out right
+    wl = make_workload(seq_lens=[900, 45, 300], query_lens=[2, 1, 1], num_q_heads=8,
+                       num_kv_heads=2, head_dim=128, block_size=16, window=0, seed=5,
+                       kv_dtype=FP8, scale=1e-3)
+    qf = wl.q.float()
+    qf[0] *= 3000.0
+    qf[1] *= 1e-3
+    qf[2, :4] *= 100.0
+    wl.q = qf.to(torch.bfloat16)
+    out = pa.decode(dev(wl), force_variant=TC)
+    check_full(wl, out, "tc query magnitudes")
+
+
+@pytest.mark.parametrize("cfg", [2, 4])
+def test_tensor_memory_kernel_full_size_sampled(cfg):
+    wl = config_workload(cfg, device="cuda:0", kv_dtype=FP8)
+    assert _variant_of(wl, force_variant=TC) == TC
+    out = pa.decode(wl, force_variant=TC)
+    torch.cuda.synchronize()
+    check_sampled(wl, out, sample_queries(wl, 32, seed=200 + cfg), f"cfg{cfg} tc full size")
