@@ -33,11 +33,15 @@ def _within_tolerance(got, ref):
     return np.all(np.isfinite(g)) and np.all(np.abs(g - r) <= ATOL + RTOL * np.abs(r))
 
 
-@pytest.mark.parametrize("kind", ["long_single_group", "gqa_ragged_mtp"])
+@pytest.mark.parametrize("kind", ["long_single_group", "gqa_ragged_mtp", "fp8_kv"])
 def test_noalloc_matches_workspace_entry_point_on_two_calls(cuda_device, kind):
     if kind == "long_single_group":
         wl = make_workload(seq_lens=[9001], query_lens=[1], num_q_heads=8, num_kv_heads=1,
                            head_dim=128, block_size=16, seed=31, device="cuda:0")
+    elif kind == "fp8_kv":
+        wl = make_workload(seq_lens=[6000, 300], query_lens=[1, 4], num_q_heads=16,
+                           num_kv_heads=2, head_dim=128, block_size=16, seed=33,
+                           device="cuda:0", kv_dtype="fp8_e4m3", q_dtype="fp8_e4m3")
     else:
         wl = make_workload(seq_lens=[3000, 777, 5120, 64], query_lens=[1, 3, 2, 1],
                            num_q_heads=32, num_kv_heads=8, head_dim=128, block_size=16,
@@ -47,12 +51,12 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(cuda_device, kind):
     assert 0 < need <= pa.PA_NOALLOC_SCRATCH_BYTES   # the split-K scratch is used
     ws = torch.empty(need, dtype=torch.uint8, device="cuda:0")
     p.workspace, p.workspace_bytes = ws.data_ptr(), need
-    ref = torch.empty_like(wl.q)
+    ref = torch.empty(wl.q.shape, dtype=torch.bfloat16, device="cuda:0")
     assert _call(pa.pa_decode, wl, p, ref) == pa.PA_OK, pa.pa_last_error()
 
     q = pa.params_for(wl)            # no workspace: the static array is used
     for _ in range(2):
-        out = torch.full_like(wl.q, float("nan"))
+        out = torch.full(wl.q.shape, float("nan"), dtype=torch.bfloat16, device="cuda:0")
         assert _call(pa.pa_decode_noalloc, wl, q, out) == pa.PA_OK, pa.pa_last_error()
         torch.cuda.synchronize()
         assert _within_tolerance(out, ref)
