@@ -282,7 +282,7 @@ int make_plan(const pa_params* p, int bs, int span, int qlen, int num_sms, int c
   in.grid_x = (int)max_parts;
   in.grid_y = p->num_kv_heads * nslab;
   in.grid_z = p->batch;
-  in.block_threads = tc ? 192 : 32 * (ncw + 1);
+  in.block_threads = tc ? 320 : 32 * (ncw + 1);
   in.smem_bytes = smem_for((int)ptok);
   in.num_sms = num_sms;
   in.ctas_per_sm = ctas_per_sm;

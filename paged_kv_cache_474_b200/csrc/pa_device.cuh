@@ -56,6 +56,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return done != 0;
 }
 
+// try_wait with a suspend-time hint: the thread sleeps until the phase
+// completes or ~1 us passes, instead of spinning through instructions other
+// warps could issue.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar), "r"(parity), "r"(1000u)
+      : "memory");
+  return done != 0;
+}
+
 // Bounded wait: spins on try_wait for at most ~kWaitCycles SM clocks (about a
 // second).  On timeout it records PA_DEV_TIMEOUT in the status word and
 // returns false; callers then stop consuming and leave the kernel cleanly.
@@ -64,7 +79,7 @@ constexpr long long kWaitCycles = 2000000000LL;
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait_sleep(bar, parity)) {
     if (clock64() - t0 > kWaitCycles) {
       atomicOr(&g_pa_status, PA_DEV_TIMEOUT);
       return false;

@@ -1237,7 +1237,7 @@ cudaError_t launch_tc_t(const DecodeArgs& a, const CUtensorMap& tk, const CUtens
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(192);
+  cfg.blockDim = dim3(320);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -1269,7 +1269,7 @@ int occupancy_tc_t(size_t smem) {
   const long long per_cta_smem = (long long)smem + (long long)fa.sharedSizeBytes + reserved;
   const int regs = ((fa.numRegs + 7) / 8) * 8;  // allocated per thread in units of 8
   int n = (int)(sm_smem / per_cta_smem);
-  n = std::min(n, sm_regs / (regs * 192));
+  n = std::min(n, sm_regs / (regs * 320));
   n = std::min(n, 512 / kTcTmemCols);  // tensor-memory columns per SM
   return std::max(n, 0);
 }

@@ -76,7 +76,7 @@ int occupancy_partition_mma(const KernelShape& k, size_t smem);
 // (FP8 caches, head_dim 128, 128-token stages).
 size_t tc_smem_bytes(int stages, int part_tokens, int block_size);
 
-// Launches the tcgen05 partition kernel (192 threads); tk / tv as for the
+// Launches the tcgen05 partition kernel (320 threads); tk / tv as for the
 // tensor-core kernel with FP8 caches.
 cudaError_t launch_partition_tc(const DecodeArgs& a, const KernelShape& k, const CUtensorMap& tk,
                                 const CUtensorMap& tv, dim3 grid, size_t smem,

@@ -21,12 +21,14 @@
 // and split the same way.  Each split doubles the MMAs of its product, which
 // the tensor cores have to spare on this HBM-bound path.
 //
-// Roles (192 threads): warp 0 copies (TMA ring), warp 1 issues the MMAs from
-// one thread and owns the tensor-memory allocation, warps 2..5 (128 threads)
+// Roles (320 threads): warp 0 copies (TMA ring), warp 1 issues the MMAs from
+// one thread and owns the tensor-memory allocation, warps 2..9 (256 threads)
 // run the softmax and accumulate O.  Warp w may only touch TMEM lanes
 // 32*(w%4)..+31, so softmax warp w owns tokens 32*(w%4)..+31 of each stage
-// (as rows of S^T) and dims 32*(w%4)..+31 (as rows of O).  Each softmax
-// warp keeps its own running max per row over its 32-token slice of every
+// (as rows of S^T) and dims 32*(w%4)..+31 (as rows of O), for half of the
+// query rows (two warps per lane quadrant, so twice the warps hide the
+// softmax's dependent chain).  Each softmax warp keeps its own running max
+// per row over its 32-token slice of every
 // stage, so no statistic crosses warps until the partition ends; the PV
 // product is therefore issued per slice (four K = 32 MMAs into four O
 // buffers), and each thread folds the four per-stage O slices into registers
@@ -96,9 +98,13 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
 
 template <int NC>
 __device__ __forceinline__ void tc_ld(uint32_t taddr, float (&v)[NC]) {
-  static_assert(NC == 8 || NC == 16, "8 or 16 columns");
+  static_assert(NC == 4 || NC == 8 || NC == 16, "4, 8 or 16 columns");
   uint32_t r[NC];
-  if constexpr (NC == 8) {
+  if constexpr (NC == 4) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(taddr));
+  } else if constexpr (NC == 8) {
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
                    "=r"(r[6]), "=r"(r[7])
@@ -143,17 +149,18 @@ __device__ __forceinline__ void tc_warp_rowmax(const float (&v)[RT], float (&out
   for (int r = 0; r < RT; ++r) out[r] = tc_unkey(__reduce_max_sync(FULL, tc_fkey(v[r])));
 }
 
-// At 128 registers four warps share an SM sub-partition's register file, so
-// two 6-warp CTAs fit an SM however their warps are spread (at 130, three
-// warps per sub-partition would leave room for one CTA).
+// At 80 registers six warps share an SM sub-partition's register file, so
+// two 10-warp CTAs fit an SM however their warps are spread.
 template <int NS, int RT>
-__global__ void __maxnreg__(128)
+__global__ void __maxnreg__(80)
     pa_partition_tc_kernel(const __grid_constant__ DecodeArgs a,
                            const __grid_constant__ CUtensorMap tmk,
                            const __grid_constant__ CUtensorMap tmv) {
   constexpr int D = 128;
   using Lt = TcLayout;
   static_assert(RT == 8 || RT == 16, "rows per CTA");
+  constexpr int NSW = 8;       // softmax warps: two per TMEM lane quadrant
+  constexpr int RW = RT / 2;   // rows per softmax warp
 
   extern __shared__ __align__(128) uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -194,11 +201,11 @@ __global__ void __maxnreg__(128)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&s_full[i]), 1);
-      mbar_init(smem_u32(&s_free[i]), 4);
-      mbar_init(smem_u32(&p_full[i]), 4);
+      mbar_init(smem_u32(&s_free[i]), NSW);
+      mbar_init(smem_u32(&p_full[i]), NSW);
     }
     mbar_init(smem_u32(o_full), 1);
-    mbar_init(smem_u32(o_free), 4);
+    mbar_init(smem_u32(o_free), NSW);
     mbar_init(smem_u32(mma_done), 1);
     fence_mbar_init();
   }
@@ -241,7 +248,7 @@ __global__ void __maxnreg__(128)
                  "r"(kTcTmemCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
-  if (warp >= 2) {
+  if (warp >= 2 && warp < 6) {
     const int t = threadIdx.x - 64;  // 0..127: (row t/8, 16-dim chunk t%8)
     const int r = t >> 3, c = t & 7;
     uint4 hi = make_uint4(0u, 0u, 0u, 0u), lo = make_uint4(0u, 0u, 0u, 0u);
@@ -305,17 +312,21 @@ __global__ void __maxnreg__(128)
       s_lo[r] = lo;
       s_hi[r] = hi;
     }
+    fence_proxy_async_smem();  // the tensor core reads Q through the async proxy
+  }
+  if (warp >= 2) {
     // P buffers start at zero: rows >= Rs are never written again
+    const int t = threadIdx.x - 64;  // 0..255
     const uint4 z = make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-      *reinterpret_cast<uint4*>(psm + (size_t)(u * 128 + t) * 16) = z;
-    fence_proxy_async_smem();  // the tensor core reads Q and P through the async proxy
+    for (int u = 0; u < 2; ++u)
+      *reinterpret_cast<uint4*>(psm + (size_t)(u * 256 + t) * 16) = z;
+    fence_proxy_async_smem();
   }
   uint32_t tmem = 0;
   if (warp != 0) {
     tc_fence_before();
-    named_bar_sync(2, 160);  // MMA and softmax warps: tensor memory, Q and P ready
+    named_bar_sync(2, 32 + 32 * NSW);  // MMA and softmax warps: tensor memory, Q and P ready
     tc_fence_after();
     tmem = s_tmem;
   }
@@ -450,20 +461,21 @@ __global__ void __maxnreg__(128)
     __syncwarp();
   } else {
     // ---------------------------- softmax warps ----------------------------
-    const int qd = warp & 3;                 // TMEM lane quadrant of this warp
-    const int tk = 32 * qd + lane;           // my token within a stage; my dim of O
+    const int qd = warp & 3;               // TMEM lane quadrant of this warp
+    const int r0w = ((warp - 2) >> 2) * RW;  // first of this warp's rows
+    const int tk = 32 * qd + lane;         // my token within a stage; my dim of O
     const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
     // (per-row scale and range live in smem: broadcast reads, no registers)
-    float m_w[RT], l_p[RT], acc[4][RT];
+    float m_w[RW], l_p[RW], acc[4][RW];
 #pragma unroll
-    for (int r = 0; r < RT; ++r) {
+    for (int r = 0; r < RW; ++r) {
       m_w[r] = kNegInf;
       l_p[r] = 0.f;
 #pragma unroll
       for (int sl = 0; sl < 4; ++sl) acc[sl][r] = 0.f;
     }
     for (int k = 0;; ++k) {
-      named_bar_sync(1, 128);  // the four softmax warps move in step
+      named_bar_sync(1, 32 * NSW);  // the softmax warps move in step
       const int s = k % NS;
       // (every decision below is warp-uniform: the tcgen05 loads are .sync.aligned)
       int c0 = -1;
@@ -479,22 +491,24 @@ __global__ void __maxnreg__(128)
       }
       if (c0 >= 0) {
         tc_fence_after();
-        float sv[RT];
-        tc_ld<RT>(tl + (k & 1) * kTcN, sv);
+        float sv[RW];
+        tc_ld<RW>(tl + (k & 1) * kTcN + r0w, sv);
         tc_wait_ld();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&s_free[k & 1]));
         const int t = c0 + tk;
-        float v[RT];
+        float v[RW];
 #pragma unroll
-        for (int r = 0; r < RT; ++r)
-          v[r] = (t >= s_lo[r] && t < s_hi[r]) ? sv[r] * (a.scale_log2 * sig_s[r]) : kNegInf;
-        float wm[RT];
-        tc_warp_rowmax<RT>(v, wm);
-        float al[RT], p[RT];
+        for (int r = 0; r < RW; ++r)
+          v[r] = (t >= s_lo[r0w + r] && t < s_hi[r0w + r])
+                     ? sv[r] * (a.scale_log2 * sig_s[r0w + r])
+                     : kNegInf;
+        float wm[RW];
+        tc_warp_rowmax<RW>(v, wm);
+        float al[RW], p[RW];
 #pragma unroll
-        for (int r = 0; r < RT; ++r) {
+        for (int r = 0; r < RW; ++r) {
           const float mn = fmaxf(m_w[r], wm[r]);
           const float mu = (mn == kNegInf) ? 0.f : mn;
           al[r] = (mn == kNegInf) ? 1.f : ex2(m_w[r] - mu);
@@ -503,18 +517,18 @@ __global__ void __maxnreg__(128)
           l_p[r] = l_p[r] * al[r] + p[r];
         }
 #pragma unroll
-        for (int r = 0; r < RT; ++r)
-          if (lane == r) alpha_s[(k & 1) * 4 * kTcN + qd * kTcN + r] = al[r];
+        for (int r = 0; r < RW; ++r)
+          if (lane == r) alpha_s[(k & 1) * 4 * kTcN + qd * kTcN + r0w + r] = al[r];
         // P^T (x 256) as hi + lo e4m3 terms, one byte per (row, token)
         uint8_t* pb = psm + (k & 1) * 2 * Lt::PB_BYTES;
 #pragma unroll
-        for (int r = 0; r < RT; r += 2) {
+        for (int r = 0; r < RW; r += 2) {
           const float x0 = p[r] * 256.f, x1 = p[r + 1] * 256.f;
           const uint32_t h = f32x2_to_e4m3x2(x0, x1);
           const uint32_t hf = e4m3x2_to_f16x2(h);
           const float2 g = __half22float2(*reinterpret_cast<const __half2*>(&hf));
           const uint32_t lw = f32x2_to_e4m3x2(x0 - g.x, x1 - g.y);
-          const uint32_t o0 = tc_sw128(r, tk), o1 = tc_sw128(r + 1, tk);
+          const uint32_t o0 = tc_sw128(r0w + r, tk), o1 = tc_sw128(r0w + r + 1, tk);
           pb[o0] = (uint8_t)(h & 0xffu);
           pb[o1] = (uint8_t)(h >> 8);
           pb[Lt::PB_BYTES + o0] = (uint8_t)(lw & 0xffu);
@@ -522,12 +536,15 @@ __global__ void __maxnreg__(128)
         }
         // V rows of tokens outside the row's union span may hold anything
         // (uninitialised cache slots, earlier stages): zero them so the PV
-        // product never multiplies a 0 weight by a NaN.
+        // product never multiplies a 0 weight by a NaN.  The two warps of a
+        // quadrant zero one half of the row each.
         if (t < ulo || t >= p1) {
           const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-          uint4* vr = reinterpret_cast<uint4*>(smem + s * Lt::STAGE_BYTES + Lt::KV_BYTES + tk * Lt::ROW);
+          uint4* vr = reinterpret_cast<uint4*>(smem + s * Lt::STAGE_BYTES + Lt::KV_BYTES +
+                                               tk * Lt::ROW) +
+                      (r0w ? 4 : 0);
 #pragma unroll
-          for (int cc = 0; cc < 8; ++cc) vr[cc] = z;
+          for (int cc = 0; cc < 4; ++cc) vr[cc] = z;
         }
         fence_proxy_async_smem();
         __syncwarp();
@@ -539,18 +556,18 @@ __global__ void __maxnreg__(128)
         const bool got = ok && __all_sync(FULL, mbar_wait(smem_u32(o_full), pk & 1));
         if (got) {
           tc_fence_after();
-          float ov[4][RT];
+          float ov[4][RW];
 #pragma unroll
-          for (int sl = 0; sl < 4; ++sl) tc_ld<RT>(tl + 2 * kTcN + sl * kTcN, ov[sl]);
+          for (int sl = 0; sl < 4; ++sl) tc_ld<RW>(tl + 2 * kTcN + sl * kTcN + r0w, ov[sl]);
           tc_wait_ld();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(o_free));
-          const float* alp = alpha_s + (pk & 1) * 4 * kTcN;
+          const float* alp = alpha_s + (pk & 1) * 4 * kTcN + r0w;
 #pragma unroll
           for (int sl = 0; sl < 4; ++sl)
 #pragma unroll
-            for (int r = 0; r < RT; ++r) acc[sl][r] = acc[sl][r] * alp[sl * kTcN + r] + ov[sl][r];
+            for (int r = 0; r < RW; ++r) acc[sl][r] = acc[sl][r] * alp[sl * kTcN + r] + ov[sl][r];
         } else {
           ok = false;
         }
@@ -560,37 +577,37 @@ __global__ void __maxnreg__(128)
 
     // ---- merge the four token slices and write the partial --------------
 #pragma unroll
-    for (int r = 0; r < RT; ++r) {
+    for (int r = 0; r < RW; ++r) {
       float ls = l_p[r];
 #pragma unroll
       for (int o = 16; o; o >>= 1) ls += __shfl_xor_sync(FULL, ls, o);
       if (lane == r) {
-        stat_m[qd * kTcN + r] = m_w[r];
-        stat_l[qd * kTcN + r] = ls;
+        stat_m[qd * kTcN + r0w + r] = m_w[r];
+        stat_l[qd * kTcN + r0w + r] = ls;
       }
     }
-    named_bar_sync(1, 128);
+    named_bar_sync(1, 32 * NSW);
 #pragma unroll
-    for (int r = 0; r < RT; ++r) {
-      if (r >= Rs) continue;
+    for (int r = 0; r < RW; ++r) {
+      const int row = r0w + r;
+      if (row >= Rs) continue;
       float M = kNegInf;
 #pragma unroll
-      for (int sl = 0; sl < 4; ++sl) M = fmaxf(M, stat_m[sl * kTcN + r]);
+      for (int sl = 0; sl < 4; ++sl) M = fmaxf(M, stat_m[sl * kTcN + row]);
       float Z = 0.f, O = 0.f;
 #pragma unroll
       for (int sl = 0; sl < 4; ++sl) {
-        const float f = (M == kNegInf) ? 0.f : ex2(stat_m[sl * kTcN + r] - M);
-        Z += f * stat_l[sl * kTcN + r];
+        const float f = (M == kNegInf) ? 0.f : ex2(stat_m[sl * kTcN + row] - M);
+        Z += f * stat_l[sl * kTcN + row];
         O += f * acc[sl][r];
       }
-      const int rr = row0 + r;
+      const int rr = row0 + row;
+      const float inv = Z > 0.f ? a.v_scale / (256.f * Z) : 0.f;
       if (nparts == 1) {
-        const float inv = Z > 0.f ? a.v_scale / (256.f * Z) : 0.f;
         const int i = rr / a.group, j = rr - (rr / a.group) * a.group;
         a.dst[((size_t)(qoff + i) * a.num_q_heads + (size_t)kvh * a.group + j) * D + tk] =
             __float2bfloat16_rn(O * inv);
       } else {
-        const float inv = Z > 0.f ? a.v_scale / (256.f * Z) : 0.f;
         const size_t base =
             ((size_t)(b * a.num_kv_heads + kvh) * a.max_parts + part) * a.max_rows + rr;
         a.ws_o[base * D + tk] = O * inv;

@@ -261,7 +261,7 @@ def test_plan_tensor_memory_variant_on_request():
                max_blocks_per_seq=512, max_span_hint=8192)
     assert plan(**gqa, **fp8).variant == pa.PA_VARIANT_MMA   # not chosen by itself
     info = plan(force_variant=pa.PA_VARIANT_TC, **gqa, **fp8)
-    assert info.variant == pa.PA_VARIANT_TC and info.block_threads == 192
+    assert info.variant == pa.PA_VARIANT_TC and info.block_threads == 320
     assert info.slab_rows == 8 and info.stages == 3
     assert info.partition_tokens % 128 == 0
     # more rows run as 8-row slabs; bf16 caches and other head dims are refused
