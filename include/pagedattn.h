@@ -79,6 +79,12 @@ extern "C" {
 #define PA_DTYPE_BF16 0
 #define PA_DTYPE_FP8_E4M3 1   /* per-tensor scaled FP8 e4m3 codes (tensor-core variant) */
 
+/* Scheduling of a call (pa_params.schedule). */
+#define PA_SCHED_STATIC 0     /* default: one CTA per fixed partition, then the reduce kernel */
+#define PA_SCHED_WORKLIST 2   /* one launch: a one-wave cooperative grid whose CTAs claim each
+                                 unit's 64-token stages from a work-list counter and merge their
+                                 own partials (PA_VARIANT_MMA only; see pa_params.schedule) */
+
 /* Kernel variants (pa_params.force_variant, pa_plan_info.variant). */
 #define PA_VARIANT_AUTO 0
 #define PA_VARIANT_FMA 1      /* CUDA-core FMA scores and PV (group x queryLen <= 4 rows) */
@@ -121,6 +127,18 @@ typedef struct pa_params {
     float q_scale;
     float k_scale;
     float v_scale;
+    /* PA_SCHED_*; 0 = PA_SCHED_STATIC.  PA_SCHED_WORKLIST (aiter PR #2914's
+     * persistent-scheduling idea, on one wave): one launch whose CTAs take a
+     * unit's stages in arrival order from a counter in the workspace and
+     * merge the unit's partials themselves after an arrival count, so no
+     * reduce kernel runs.  It needs PA_VARIANT_MMA and a grid that
+     * fits the GPU at once (PA_ERR_UNSUPPORTED otherwise, PA_ERR_CUDA if the
+     * cooperative launch is refused).  The counters are tagged with a
+     * per-call epoch and need no initialisation; calls that share a
+     * workspace must not overlap.  Results can differ from the static
+     * schedule's in the last bits (the stages' grouping depends on timing),
+     * and it measures slower on the named workloads, so it is opt-in. */
+    int schedule;
 } pa_params;
 
 /* What the dispatcher chose for a call (pa_plan). */
@@ -138,6 +156,7 @@ typedef struct pa_plan_info {
     size_t smem_bytes;
     size_t workspace_bytes;  /* 0 when one_shot */
     int num_sms, ctas_per_sm;
+    int worklist;            /* 1: work-list schedule (no reduce launch) */
 } pa_plan_info;
 
 /*

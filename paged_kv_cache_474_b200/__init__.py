@@ -37,6 +37,9 @@ PA_VARIANT_TC = 3
 PA_DTYPE_BF16 = 0
 PA_DTYPE_FP8_E4M3 = 1
 
+PA_SCHED_STATIC = 0
+PA_SCHED_WORKLIST = 2
+
 
 class pa_params(ctypes.Structure):
     _fields_ = [
@@ -59,6 +62,7 @@ class pa_params(ctypes.Structure):
         ("q_scale", ctypes.c_float),
         ("k_scale", ctypes.c_float),
         ("v_scale", ctypes.c_float),
+        ("schedule", ctypes.c_int),
     ]
 
 
@@ -80,6 +84,7 @@ class pa_plan_info(ctypes.Structure):
         ("workspace_bytes", ctypes.c_size_t),
         ("num_sms", ctypes.c_int),
         ("ctas_per_sm", ctypes.c_int),
+        ("worklist", ctypes.c_int),
     ]
 
     def as_dict(self):
@@ -214,7 +219,8 @@ def make_params(*, batch, num_q_heads, num_kv_heads, head_dim, num_blocks,
                 max_blocks_per_seq, max_span_hint=0, max_query_len_hint=0,
                 windows=None, workspace=None, force_variant=PA_VARIANT_AUTO,
                 force_partitions=0, q_dtype=PA_DTYPE_BF16, kv_dtype=PA_DTYPE_BF16,
-                q_scale=0.0, k_scale=0.0, v_scale=0.0) -> pa_params:
+                q_scale=0.0, k_scale=0.0, v_scale=0.0,
+                schedule=PA_SCHED_STATIC) -> pa_params:
     p = pa_params()
     p.batch = int(batch)
     p.num_q_heads = int(num_q_heads)
@@ -235,6 +241,7 @@ def make_params(*, batch, num_q_heads, num_kv_heads, head_dim, num_blocks,
     p.q_scale = float(q_scale)
     p.k_scale = float(k_scale)
     p.v_scale = float(v_scale)
+    p.schedule = int(schedule)
     return p
 
 
@@ -253,7 +260,7 @@ def pa_extents_host(seq_lens, query_lens, window=0, windows=None):
 
 
 def params_for(wl, *, workspace=None, hints=True, force_variant=PA_VARIANT_AUTO,
-               force_partitions=0) -> pa_params:
+               force_partitions=0, schedule=PA_SCHED_STATIC) -> pa_params:
     """pa_params for a ``workloads.Workload`` (host hints from its lengths)."""
     span = qlen = 0
     if hints:
@@ -271,7 +278,8 @@ def params_for(wl, *, workspace=None, hints=True, force_variant=PA_VARIANT_AUTO,
                        kv_dtype=PA_DTYPE_FP8_E4M3 if wl.kv_fp8 else PA_DTYPE_BF16,
                        q_scale=wl.q_scale if wl.q_fp8 else 0.0,
                        k_scale=wl.k_scale if wl.kv_fp8 else 0.0,
-                       v_scale=wl.v_scale if wl.kv_fp8 else 0.0)
+                       v_scale=wl.v_scale if wl.kv_fp8 else 0.0,
+                       schedule=schedule)
 
 
 def alloc_workspace(params: pa_params, kv_block_size: int, device="cuda"):
@@ -286,17 +294,18 @@ def alloc_workspace(params: pa_params, kv_block_size: int, device="cuda"):
 
 
 def decode(wl, *, out=None, workspace=None, hints=True, force_variant=PA_VARIANT_AUTO,
-           force_partitions=0, stream=None):
+           force_partitions=0, schedule=PA_SCHED_STATIC, stream=None):
     """Runs pa_decode on a device-resident ``Workload``; returns dst (bf16
     [sum(queryLens), H_q, D]).  Allocates the workspace when none is given."""
     import torch
     p = params_for(wl, workspace=workspace, hints=hints, force_variant=force_variant,
-                   force_partitions=force_partitions)
+                   force_partitions=force_partitions, schedule=schedule)
     if workspace is None:
         # size the workspace from the real extents even when the call itself
         # runs without hints (pa_decode then reads the lengths itself)
         sizing = p if hints else params_for(wl, force_variant=force_variant,
-                                            force_partitions=force_partitions)
+                                            force_partitions=force_partitions,
+                                            schedule=schedule)
         workspace = alloc_workspace(sizing, wl.block_size, device=wl.q.device)
         if workspace is not None:
             p.workspace = workspace.data_ptr()

@@ -14,6 +14,7 @@
 // the one-shot path: the kernel writes dst itself, with no workspace and no
 // reduce (aiter PR #2914 "Pa gluon swa mtp opt", one_shot).
 #include <algorithm>
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -105,6 +106,8 @@ int check_params(const pa_params* p, int bs) {
   if (p->max_span_hint < 0 || p->max_query_len_hint < 0)
     return fail(PA_ERR_ARG, "hints must be >= 0");
   if (p->force_partitions < 0) return fail(PA_ERR_ARG, "force_partitions must be >= 0");
+  if (p->schedule != PA_SCHED_STATIC && p->schedule != PA_SCHED_WORKLIST)
+    return fail(PA_ERR_ARG, "unknown schedule %d", p->schedule);
   if (p->force_variant != PA_VARIANT_AUTO && p->force_variant != PA_VARIANT_FMA &&
       p->force_variant != PA_VARIANT_MMA && p->force_variant != PA_VARIANT_TC)
     return fail(PA_ERR_ARG, "unknown force_variant %d", p->force_variant);
@@ -153,7 +156,7 @@ int cached_occupancy(bool mma, const pa::KernelShape& k, size_t smem) {
 struct Plan {
   pa_plan_info info;
   pa::KernelShape shape;
-  size_t lse_bytes, o_bytes;
+  size_t lse_bytes, o_bytes, ctr_bytes;
 };
 
 // span: longest union span over rows; qlen: longest queryLen.
@@ -286,11 +289,23 @@ int make_plan(const pa_params* p, int bs, int span, int qlen, int num_sms, int c
   in.smem_bytes = smem_for((int)ptok);
   in.num_sms = num_sms;
   in.ctas_per_sm = ctas_per_sm;
+  if (p->schedule == PA_SCHED_WORKLIST) {
+    const long long ctas = (long long)in.grid_x * in.grid_y * in.grid_z;
+    if (variant != PA_VARIANT_MMA || ctas > slots)
+      return fail(PA_ERR_UNSUPPORTED,
+                  "the work-list schedule needs the MMA variant and a one-wave grid "
+                  "(%lld CTAs, %lld slots)",
+                  ctas, slots);
+  }
   if (!in.one_shot) {
     const size_t partials = (size_t)p->batch * p->num_kv_heads * max_parts * rmax;
     pl.lse_bytes = align256(partials * sizeof(float));
     pl.o_bytes = align256(partials * p->head_dim * sizeof(float));
-    in.workspace_bytes = pl.lse_bytes + pl.o_bytes;
+    in.worklist = p->schedule == PA_SCHED_WORKLIST;
+    // two epoch-tagged counters per unit: stages handed out, partials published
+    if (in.worklist)
+      pl.ctr_bytes = align256(2 * (size_t)in.grid_z * in.grid_y * sizeof(uint64_t));
+    in.workspace_bytes = pl.lse_bytes + pl.o_bytes + pl.ctr_bytes;
   }
   *out = pl;
   return PA_OK;
@@ -434,6 +449,15 @@ int decode_impl(void* dst, const void* q, const void* kCache, const void* vCache
     char* ws = static_cast<char*>(p->workspace);
     a.ws_lse = reinterpret_cast<float*>(ws);
     a.ws_o = reinterpret_cast<float*>(ws + pl.lse_bytes);
+    if (in.worklist) {
+      static std::atomic<unsigned int> epochs{0};
+      unsigned int e = ++epochs;
+      if (e == 0) e = ++epochs;  // 0 is never a live epoch
+      a.worklist = 1;
+      a.epoch = e;
+      a.stage_ctr = reinterpret_cast<unsigned long long*>(ws + pl.lse_bytes + pl.o_bytes);
+      a.done = a.stage_ctr + (size_t)in.grid_z * in.grid_y;
+    }
   }
   // FP8 scales: q_scale * k_scale multiplies every score, v_scale every output
   double sc = (double)scale * 1.4426950408889634;
@@ -483,7 +507,7 @@ int decode_impl(void* dst, const void* q, const void* kCache, const void* vCache
   }
   if (e == cudaSuccess && ev1) e = cudaEventRecord(ev1, stream);
   if (e != cudaSuccess) return fail(PA_ERR_CUDA, "partition kernel launch: %s", cudaGetErrorString(e));
-  if (!in.one_shot) {
+  if (!in.one_shot && !a.worklist) {
     e = pa::launch_reduce(a, stream);
     if (e != cudaSuccess) return fail(PA_ERR_CUDA, "reduce kernel launch: %s", cudaGetErrorString(e));
   }

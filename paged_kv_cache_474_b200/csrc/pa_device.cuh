@@ -88,6 +88,48 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   return true;
 }
 
+// Epoch-tagged counters of the work-list schedule live in the caller's
+// workspace, which is never initialised: the high 32 bits hold the epoch of
+// the call that last touched the counter, the low 32 bits its count.  The
+// first touch of a call resets a stale counter (one CAS: if it fails, another
+// CTA of the same call reset or advanced it first, so it is current).
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void epoch_touch(unsigned long long* c, unsigned int epoch) {
+  const unsigned long long cur = ld_acquire_u64(c);
+  if ((unsigned int)(cur >> 32) != epoch) atomicCAS(c, cur, (unsigned long long)epoch << 32);
+}
+
+// First stage index of a claim from the counter's previous value v (an
+// atomicAdd's result); INT_MAX (stop) if the counter was not this call's,
+// which cannot happen after epoch_touch.
+__device__ __forceinline__ int claim_value(unsigned long long v, unsigned int epoch) {
+  return (unsigned int)(v >> 32) == epoch ? (int)(unsigned int)v : 0x7fffffff;
+}
+
+__device__ __forceinline__ void epoch_arrive(unsigned long long* c, unsigned int epoch) {
+  epoch_touch(c, epoch);
+  atomicAdd(c, 1ull);
+}
+
+// Bounded wait (same limit as mbar_wait) for `target` arrivals of this epoch.
+__device__ __forceinline__ bool epoch_wait(const unsigned long long* c, unsigned int epoch,
+                                           unsigned int target) {
+  const long long t0 = clock64();
+  while (true) {
+    const unsigned long long v = ld_acquire_u64(c);
+    if ((unsigned int)(v >> 32) == epoch && (unsigned int)v >= target) return true;
+    if (clock64() - t0 > kWaitCycles) {
+      atomicOr(&g_pa_status, PA_DEV_TIMEOUT);
+      return false;
+    }
+  }
+}
+
 // 1-D bulk copy global -> shared (the TMA engine's non-tensor path); completes
 // `bytes` transaction bytes on `bar`.  Addresses 16-byte aligned, bytes a
 // multiple of 16.

@@ -469,10 +469,98 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
   return y;
 }
 
+struct LseAcc {
+  float m, z;
+  float4 o;
+};
+
+// (m, z, o) += (m2, z2, o2) with the larger maximum kept; -inf maxima weigh 0.
+__device__ __forceinline__ void lse_merge(LseAcc& x, float m2, float z2, float4 o2) {
+  const float mn = fmaxf(x.m, m2);
+  const float f1 = mn == kNegInf ? 0.f : ex2(x.m - mn);
+  const float f2 = mn == kNegInf ? 0.f : ex2(m2 - mn);
+  x.z = x.z * f1 + z2 * f2;
+  x.o.x = x.o.x * f1 + o2.x * f2;
+  x.o.y = x.o.y * f1 + o2.y * f2;
+  x.o.z = x.o.z * f1 + o2.z * f2;
+  x.o.w = x.o.w * f1 + o2.w * f2;
+  x.m = mn;
+}
+
+// ---------------------------------------------------------------------------
+// Work-list merge (the reduce below, done by the unit's own CTAs).  Used by
+// the work-list schedule, whose one-wave grid is launched cooperatively, so
+// every CTA of a unit is resident: each CTA publishes its partial (fence, then
+// an epoch-tagged arrival), waits until all nparts partials of its unit have
+// arrived, then merges a share of the unit's outputs -- one warp per (row,
+// 4 dims), its lanes striding over the partials with a running log-sum-exp
+// and a butterfly merge at the end.  Partials are read through L2 (ld.cg):
+// other SMs wrote them during this kernel.
+// ---------------------------------------------------------------------------
+template <int D>
+__device__ __noinline__ void merge_unit_partials(const DecodeArgs& a, int b, int kvh, int part,
+                                                 int nparts, int row0, int Rs, int qoff) {
+  __shared__ int s_go;
+  __threadfence();
+  __syncthreads();
+  unsigned long long* cnt = a.done + (size_t)blockIdx.z * gridDim.y + blockIdx.y;
+  if (threadIdx.x == 0) {
+    epoch_arrive(cnt, a.epoch);
+    s_go = epoch_wait(cnt, a.epoch, (unsigned)nparts);
+    __threadfence();
+  }
+  __syncthreads();
+  if (!s_go) return;
+  constexpr int C4 = D / 4;
+  constexpr int BATCH = 4;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nw = blockDim.x >> 5;
+  const size_t ubase = (size_t)(b * a.num_kv_heads + kvh) * a.max_parts;
+  for (int j = part * nw + warp; j < Rs * C4; j += nparts * nw) {
+    const int r = j / C4, c4 = j - (j / C4) * C4;
+    const int rr = row0 + r;
+    LseAcc acc{kNegInf, 0.f, make_float4(0.f, 0.f, 0.f, 0.f)};
+    for (int p0 = lane; p0 < nparts; p0 += 32 * BATCH) {
+      float l[BATCH];
+      float4 o[BATCH];
+#pragma unroll
+      for (int u = 0; u < BATCH; ++u) {
+        const int p = p0 + 32 * u;
+        const size_t base = (ubase + p) * a.max_rows + rr;
+        l[u] = p < nparts ? __ldcg(a.ws_lse + base) : kNegInf;
+        o[u] = p < nparts ? __ldcg(reinterpret_cast<const float4*>(a.ws_o + base * D) + c4)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < BATCH; ++u) lse_merge(acc, l[u], 1.f, o[u]);
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) {
+      const float m2 = __shfl_xor_sync(FULL, acc.m, off);
+      const float z2 = __shfl_xor_sync(FULL, acc.z, off);
+      float4 o2;
+      o2.x = __shfl_xor_sync(FULL, acc.o.x, off);
+      o2.y = __shfl_xor_sync(FULL, acc.o.y, off);
+      o2.z = __shfl_xor_sync(FULL, acc.o.z, off);
+      o2.w = __shfl_xor_sync(FULL, acc.o.w, off);
+      lse_merge(acc, m2, z2, o2);
+    }
+    if (lane == 0) {
+      const float inv = acc.z > 0.f ? 1.f / acc.z : 0.f;
+      const int i = rr / a.group, jj = rr - (rr / a.group) * a.group;
+      __nv_bfloat16* dp =
+          a.dst + ((size_t)(qoff + i) * a.num_q_heads + (size_t)kvh * a.group + jj) * D + c4 * 4;
+      *reinterpret_cast<__nv_bfloat162*>(dp) = __floats2bfloat162_rn(acc.o.x * inv, acc.o.y * inv);
+      *reinterpret_cast<__nv_bfloat162*>(dp + 2) =
+          __floats2bfloat162_rn(acc.o.z * inv, acc.o.w * inv);
+    }
+  }
+}
+
 // Register caps keep 4 (one n-tile) or 3 (two n-tiles) warps per SM
 // sub-partition, so two CTAs fit per SM; head_dim 256 runs one CTA per SM
 // (its 192 KB ring) and takes the larger cap for its wider accumulators.
-template <int D, int NCW, int NSTAGE, int N8, bool F8>
+template <int D, int NCW, int NSTAGE, int N8, bool F8, bool WL>
 __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
     pa_partition_mma_kernel(const __grid_constant__ DecodeArgs a,
                             const __grid_constant__ CUtensorMap tmk,
@@ -497,6 +585,7 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
 
   __shared__ int s_qoff;
   __shared__ float s_fac[NCW][64], s_rowm[64], s_rowz[64];  // warp-merge factors (rows <= 64)
+  __shared__ int s_c0[WL ? NSTAGE : 1];  // work list: each slot's first token; -1: stop
 
   // Nothing here depends on the inputs: set up the pipeline while the
   // previous kernel on the stream may still be finishing (this kernel is
@@ -518,7 +607,7 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
   // A row without a window starts its partitions at token 0, so the copy warp
   // can fetch the partition's block-table slice while the lengths are still
   // in flight (entries past the row's last block are read but never used).
-  const bool spec_table = (a.windows == nullptr && a.window == 0);
+  const bool spec_table = (!WL && a.windows == nullptr && a.window == 0);
   if (warp == 0 && spec_table) {
     const int sj0 = (part * a.part_tokens) >> a.block_shift;
     const int sn = min(a.part_tokens / a.block_size + 2, a.max_blocks_per_seq - sj0);
@@ -542,8 +631,10 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
   const int row0 = slab * a.slab_rows;
   if (row0 >= R || part >= nparts) return;
   const int Rs = min(a.slab_rows, R - row0);
+  // Static schedule: this CTA's partition [p0, p1).  Work list: any stage of
+  // the unit's span [A, S), so tokens are masked only at the span's ends.
   const int p0 = A + part * a.part_tokens;
-  const int p1 = min(S, p0 + a.part_tokens);
+  const int p1 = WL ? S : min(S, p0 + a.part_tokens);
   const int nst = (p1 - p0 + TS - 1) / TS;
   const int jb0 = p0 >> a.block_shift;
   const int nbt = ((p1 - 1) >> a.block_shift) - jb0 + 1;
@@ -565,29 +656,84 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
 
   if (warp == 0) {
     // ------------------------------ copy warp ------------------------------
-    // This warp alone reads the partition's block-table slice, so the first
-    // copies go out without waiting for the compute warps' prologue.  (With
-    // spec_table the slice is already in smem: same start, same lanes.)
-    for (int i = lane; i < nbt; i += 32) {
-      int phys = spec_table ? bt_s[i] : a.block_tables[(size_t)b * a.max_blocks_per_seq + jb0 + i];
-      if (phys < 0 || phys >= a.num_blocks) {
-        atomicOr(&g_pa_status, PA_DEV_BAD_BLOCK);
-        phys = -1;
+    // Static schedule: this warp alone reads the partition's block-table
+    // slice, so the first copies go out without waiting for the compute
+    // warps' prologue (with spec_table the slice is already in smem: same
+    // start, same lanes).  Work list: the unit's CTAs claim its 64-token
+    // stages from an epoch-tagged counter in the workspace, the first claim a
+    // ring's worth, later claims one stage, each issued a stage ahead; the
+    // copy warp reads each claimed stage's block-table entries itself.
+    // The work list also passes each stage's first token through s_c0 before
+    // the stage's arrival, and a last stage with s_c0 = -1 tells the compute
+    // warps to stop (the static schedule's warps count its stages).
+    if constexpr (!WL) {
+      for (int i = lane; i < nbt; i += 32) {
+        int phys =
+            spec_table ? bt_s[i] : a.block_tables[(size_t)b * a.max_blocks_per_seq + jb0 + i];
+        if (phys < 0 || phys >= a.num_blocks) {
+          atomicOr(&g_pa_status, PA_DEV_BAD_BLOCK);
+          phys = -1;
+        }
+        bt_s[i] = phys;
       }
-      bt_s[i] = phys;
     }
     __syncwarp();
     const int nbox = TS / BR;
     const int nitem = nbox * 2;  // (box, K/V) per lane
-    int issued = 0;
-    for (int k = 0; k < nst; ++k) {
+    unsigned long long* ctr = nullptr;
+    unsigned long long pend = 0;  // lane 0: the claim in flight (raw counter value)
+    int cur = 0, left = 0;        // claimed stages not yet issued: cur, cur+1, ...
+    if constexpr (WL) {
+      ctr = a.stage_ctr + (size_t)blockIdx.z * gridDim.y + blockIdx.y;
+      int first = 0;
+      if (lane == 0) {
+        epoch_touch(ctr, a.epoch);
+        first = claim_value(atomicAdd(ctr, (unsigned long long)NSTAGE), a.epoch);
+      }
+      cur = __shfl_sync(FULL, first, 0);
+      left = NSTAGE;
+    }
+    const int nst_unit = (S - A + TS - 1) / TS;
+    int k = 0;
+    bool ok = true;
+    for (;; ++k) {
+      int c0;
+      int phys_w = -1;  // work list: this lane's box block, read for this stage
+      if constexpr (WL) {
+        if (left == 0) {
+          int v = 0;
+          if (lane == 0) v = claim_value(pend, a.epoch);
+          cur = __shfl_sync(FULL, v, 0);
+          left = 1;
+        }
+        const int st = cur++;
+        --left;
+        if (st >= nst_unit) break;
+        if (left == 0 && lane == 0) pend = atomicAdd(ctr, 1ull);
+        c0 = A + st * TS;
+        if (lane < nitem) {
+          const int bt0 = c0 + (lane >> 1) * BR;
+          if (bt0 < S && bt0 + BR > ulo) {
+            phys_w = a.block_tables[(size_t)b * a.max_blocks_per_seq + (bt0 >> a.block_shift)];
+            if (phys_w < 0 || phys_w >= a.num_blocks) {
+              atomicOr(&g_pa_status, PA_DEV_BAD_BLOCK);
+              phys_w = -1;
+            }
+          }
+        }
+      } else {
+        if (k >= nst) break;
+        c0 = p0 + k * TS;
+      }
       const int s = k % NSTAGE;
       if (k >= NSTAGE) {
         bool got = true;
         if (lane == 0) got = mbar_wait(smem_u32(&bars[NSTAGE + s]), ((k / NSTAGE) - 1) & 1);
-        if (!__shfl_sync(FULL, got, 0)) break;
+        if (!__shfl_sync(FULL, got, 0)) {
+          ok = false;
+          break;
+        }
       }
-      const int c0 = p0 + k * TS;
       const int ta = max(c0, ulo), te = min(c0 + TS, p1);
       bool mine = false;
       uint32_t dst = 0;
@@ -598,7 +744,7 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
         const int bt0 = c0 + j * BR;
         if (bt0 + BR > ta && bt0 < te) {
           const int jj = bt0 >> a.block_shift;
-          const int phys = bt_s[jj - jb0];
+          const int phys = WL ? phys_w : bt_s[jj - jb0];
           if (phys >= 0) {
             mine = true;
             y = (phys * a.num_kv_heads + kvh) * a.block_size + (bt0 - (jj << a.block_shift));
@@ -607,17 +753,30 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
         }
       }
       const uint32_t nload = __popc(__ballot_sync(FULL, mine));
-      if (lane == 0) mbar_arrive_expect_tx(smem_u32(&bars[s]), nload * box_bytes);
+      if (lane == 0) {
+        if constexpr (WL) s_c0[s] = c0;
+        mbar_arrive_expect_tx(smem_u32(&bars[s]), nload * box_bytes);
+      }
       __syncwarp();
       if (mine)
         tma_load_3d(smem_u32(smem) + dst, isv ? static_cast<const void*>(&tmv)
                                               : static_cast<const void*>(&tmk),
                     0, y, 0, smem_u32(&bars[s]));
-      issued = k + 1;
+    }
+    const int issued = k;
+    if (WL && ok && lane == 0) {
+      // the stop stage: its slot last held stage issued - NSTAGE
+      const int s = issued % NSTAGE;
+      bool got = true;
+      if (issued >= NSTAGE) got = mbar_wait(smem_u32(&bars[NSTAGE + s]), ((issued / NSTAGE) - 1) & 1);
+      if (got) {
+        s_c0[s] = -1;
+        mbar_arrive(smem_u32(&bars[s]));
+      }
     }
     if (lane == 0) {
-      for (int k = max(0, issued - NSTAGE); k < issued; ++k)
-        mbar_wait(smem_u32(&bars[k % NSTAGE]), (k / NSTAGE) & 1);
+      for (int kk = max(0, issued - NSTAGE + (WL ? 1 : 0)); kk < issued; ++kk)
+        mbar_wait(smem_u32(&bars[kk % NSTAGE]), (kk / NSTAGE) & 1);
     }
     __syncwarp();
   } else {
@@ -704,13 +863,18 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
 #pragma unroll
     for (int n = 0; n < N8; ++n) m_r[n][0] = m_r[n][1] = kNegInf, l_r[n][0] = l_r[n][1] = 0.f;
 
-    for (int k = 0; k < nst; ++k) {
+    const int kend = WL ? INT_MAX : nst;
+    for (int k = 0; k < kend; ++k) {
       const int s = k % NSTAGE;
       const bool got = mbar_wait(smem_u32(&bars[s]), (k / NSTAGE) & 1);
       if (!__all_sync(FULL, got)) break;
+      int c0 = p0 + k * TS;
+      if constexpr (WL) {
+        c0 = s_c0[s];
+        if (c0 < 0) break;
+      }
       const uint32_t Ks = smem_u32(smem + s * T::STAGE_BYTES);
       const uint32_t Vs = Ks + T::KV_BYTES;
-      const int c0 = p0 + k * TS;
       const bool all_valid = (c0 >= lo_max) && (c0 + TS <= hi_min);
       const bool boundary = (c0 < ulo) || (c0 + TS > p1);
 
@@ -959,6 +1123,8 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
       if (c4 == 0) a.ws_lse[base] = Z > 0.f ? s_rowm[r] + lg2(Z) : kNegInf;
     }
   }
+  if constexpr (WL)
+    if (nparts > 1) merge_unit_partials<D>(a, b, kvh, part, nparts, row0, Rs, qoff);
 }
 
 // ---------------------------------------------------------------------------
@@ -979,24 +1145,6 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
 // while the partition kernel drains and waits on griddepcontrol before
 // reading.
 // ---------------------------------------------------------------------------
-struct LseAcc {
-  float m, z;
-  float4 o;
-};
-
-// (m, z, o) += (m2, z2, o2) with the larger maximum kept; -inf maxima weigh 0.
-__device__ __forceinline__ void lse_merge(LseAcc& x, float m2, float z2, float4 o2) {
-  const float mn = fmaxf(x.m, m2);
-  const float f1 = mn == kNegInf ? 0.f : ex2(x.m - mn);
-  const float f2 = mn == kNegInf ? 0.f : ex2(m2 - mn);
-  x.z = x.z * f1 + z2 * f2;
-  x.o.x = x.o.x * f1 + o2.x * f2;
-  x.o.y = x.o.y * f1 + o2.y * f2;
-  x.o.z = x.o.z * f1 + o2.z * f2;
-  x.o.w = x.o.w * f1 + o2.w * f2;
-  x.m = mn;
-}
-
 template <int D, int DSPLIT>
 __global__ void __launch_bounds__(512) pa_reduce_kernel(const __grid_constant__ DecodeArgs a) {
   constexpr int DC = D / DSPLIT;  // dims per CTA
@@ -1197,7 +1345,8 @@ int occupancy_fma_t(size_t smem) {
 template <int D, int NCW, int NSTAGE, int N8, bool F8>
 cudaError_t launch_mma_t(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv,
                          dim3 grid, size_t smem, cudaStream_t stream) {
-  auto kern = pa_partition_mma_kernel<D, NCW, NSTAGE, N8, F8>;
+  auto kern = a.worklist ? pa_partition_mma_kernel<D, NCW, NSTAGE, N8, F8, true>
+                         : pa_partition_mma_kernel<D, NCW, NSTAGE, N8, F8, false>;
   cudaError_t e = ensure_smem_attrs(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   // Programmatic stream serialization: CTAs may start (and set up their
@@ -1208,17 +1357,19 @@ cudaError_t launch_mma_t(const DecodeArgs& a, const CUtensorMap& tk, const CUten
   cfg.blockDim = dim3(32 * (NCW + 1));
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeCooperative;  // work list: every CTA resident at once
+  attr[1].val.cooperative = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = a.worklist ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kern, a, tk, tv);
 }
 
 template <int D, int NCW, int NSTAGE, int N8, bool F8>
 int occupancy_mma_t(size_t smem) {
-  auto kern = pa_partition_mma_kernel<D, NCW, NSTAGE, N8, F8>;
+  auto kern = pa_partition_mma_kernel<D, NCW, NSTAGE, N8, F8, false>;
   if (ensure_smem_attrs(reinterpret_cast<const void*>(kern), smem) != cudaSuccess) return 0;
   int n = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, 32 * (NCW + 1), smem) != cudaSuccess)

@@ -37,6 +37,13 @@ struct DecodeArgs {
   int max_rows;     // rows per unit the workspace holds
   int slab_rows;    // rows one CTA handles
   int num_slabs;    // CTAs per unit along grid.y (grid.y = H_kv * num_slabs)
+  // Work-list schedule (tensor-core kernel, one-wave cooperative grid): a
+  // unit's CTAs claim its 64-token stages from a counter and merge their own
+  // partials instead of a reduce kernel.
+  int worklist;
+  unsigned int epoch;             // this call's tag for the counters below
+  unsigned long long* stage_ctr;  // [B][grid.y] next stage to hand out
+  unsigned long long* done;       // [B][grid.y] partials published
 };
 
 // Compile-time shape of a partition-kernel instance.
@@ -69,6 +76,7 @@ size_t mma_smem_bytes(int head_dim, int elem_bytes, int stages, int part_tokens,
 cudaError_t launch_partition_mma(const DecodeArgs& a, const KernelShape& k, const CUtensorMap& tk,
                                  const CUtensorMap& tv, dim3 grid, size_t smem,
                                  cudaStream_t stream);
+// (a.worklist launches cooperatively: every CTA of the grid is resident at once.)
 
 int occupancy_partition_mma(const KernelShape& k, size_t smem);
 

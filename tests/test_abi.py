@@ -60,6 +60,8 @@ def call(p, bs=16, window=0, scale=0.125, ptrs=16):
     (dict(max_span_hint=-3), pa.PA_ERR_ARG),
     (dict(force_partitions=-1), pa.PA_ERR_ARG),
     (dict(force_variant=7), pa.PA_ERR_ARG),
+    (dict(schedule=1), pa.PA_ERR_ARG),
+    (dict(schedule=3), pa.PA_ERR_ARG),
     (dict(force_variant=4), pa.PA_ERR_ARG),
 ])
 def test_invalid_params_are_rejected_on_the_host(kw, code):
@@ -276,3 +278,24 @@ def test_plan_tensor_memory_variant_on_request():
                     max_blocks_per_seq=8192, max_span_hint=131072,
                     force_variant=pa.PA_VARIANT_TC, **fp8)
     assert long_row.variant == pa.PA_VARIANT_TC and long_row.partition_tokens % 128 == 0
+
+
+def test_plan_work_list_schedule():
+    long_row = dict(batch=1, num_q_heads=8, num_kv_heads=1, head_dim=128, num_blocks=8193,
+                    max_blocks_per_seq=8192, max_span_hint=131072)
+    static = plan(**long_row)
+    assert not static.worklist
+    wl = plan(schedule=pa.PA_SCHED_WORKLIST, **long_row)
+    assert wl.worklist and wl.grid_x * wl.grid_y * wl.grid_z <= 148 * 2
+    align = lambda x: (x + 255) // 256 * 256
+    assert wl.workspace_bytes == static.workspace_bytes + align(2 * 1 * 1 * 8)
+    # more CTAs than one wave, or a variant other than MMA: refused
+    many = dict(batch=32, num_q_heads=32, num_kv_heads=8, head_dim=128, num_blocks=20000,
+                max_blocks_per_seq=512, max_span_hint=8192)
+    rc, _ = pa.pa_plan(base_params(schedule=pa.PA_SCHED_WORKLIST, **many), 16, 148, 2)
+    assert rc == pa.PA_ERR_UNSUPPORTED
+    rc, _ = pa.pa_plan(base_params(schedule=pa.PA_SCHED_WORKLIST, force_variant=pa.PA_VARIANT_FMA,
+                                   **long_row), 16, 148, 2)
+    assert rc == pa.PA_ERR_UNSUPPORTED
+    one_shot = plan(schedule=pa.PA_SCHED_WORKLIST, max_span_hint=50)
+    assert one_shot.one_shot and not one_shot.worklist and one_shot.workspace_bytes == 0

@@ -347,3 +347,78 @@ def test_unreachable_blocks_match_oracle():
             W = None if ws is None else torch.tensor(ws, dtype=torch.int32, device="cuda:0")
             got = pa.unreachable_blocks(S, L, bs, w, W).cpu().numpy()
             assert np.array_equal(got, oracle.unreachable_blocks(s, l, bs, w, ws))
+
+
+# ------------------------------------------------- work-list schedule
+def _wl_case(case):
+    if case == "long":
+        return make_workload(seq_lens=[9001], query_lens=[1], num_q_heads=8, num_kv_heads=1,
+                             head_dim=128, block_size=16, seed=41)
+    if case == "rows":
+        return make_workload(seq_lens=[5000, 333, 77, 1], query_lens=[1, 3, 2, 1], num_q_heads=8,
+                             num_kv_heads=2, head_dim=128, block_size=16, seed=42)
+    if case == "windows":
+        return make_workload(seq_lens=[6000, 2500, 300], query_lens=[2, 1, 5], num_q_heads=8,
+                             num_kv_heads=2, head_dim=64, block_size=64, windows=[1000, 0, 16],
+                             seed=43)
+    if case == "slabs":
+        return make_workload(seq_lens=[3000, 1200], query_lens=[5, 2], num_q_heads=32,
+                             num_kv_heads=2, head_dim=128, block_size=16, seed=44)
+    if case == "fp8":
+        return make_workload(seq_lens=[7000, 900], query_lens=[1, 4], num_q_heads=16,
+                             num_kv_heads=2, head_dim=128, block_size=1024, seed=45,
+                             kv_dtype="fp8_e4m3")
+    if case == "d256":
+        return make_workload(seq_lens=[4000, 100], query_lens=[1, 2], num_q_heads=16,
+                             num_kv_heads=2, head_dim=256, block_size=16, seed=46)
+    raise ValueError(case)
+
+
+@pytest.mark.parametrize("case", ["long", "rows", "windows", "slabs", "fp8", "d256"])
+def test_work_list_schedule_matches_oracle(case):
+    wl = _wl_case(case)
+    d = dev(wl)
+    _, info = pa.pa_plan(pa.params_for(d, schedule=pa.PA_SCHED_WORKLIST), wl.block_size)
+    assert info.max_partitions > 1 and info.worklist
+    out = pa.decode(d, schedule=pa.PA_SCHED_WORKLIST)
+    check_full(wl, out, f"work list {case}")
+
+
+@pytest.mark.parametrize("parts", [2, 7, 30])
+def test_work_list_schedule_with_forced_partitions(parts):
+    # more CTAs per unit than stages for the short rows: some claim nothing
+    wl = _wl_case("rows")
+    out = pa.decode(dev(wl), schedule=pa.PA_SCHED_WORKLIST, force_partitions=parts)
+    check_full(wl, out, f"work list parts={parts}")
+
+
+@pytest.mark.parametrize("fill", [0x00, 0xFF, "random", "reuse"])
+def test_work_list_workspace_needs_no_initialisation(fill):
+    # the counters are epoch-tagged: stale, garbage or reused workspaces give
+    # the same result as a fresh one
+    wl = _wl_case("rows")
+    d = dev(wl)
+    p = pa.params_for(d, schedule=pa.PA_SCHED_WORKLIST)
+    ws = pa.alloc_workspace(p, wl.block_size)
+    if fill == "random":
+        ws.copy_(torch.randint(0, 256, ws.shape, dtype=torch.uint8, device=ws.device))
+    elif fill != "reuse":
+        ws.fill_(fill)
+    ref = oracle.decode(problem(wl))
+    for _ in range(3 if fill == "reuse" else 1):
+        out = pa.decode(d, workspace=ws, schedule=pa.PA_SCHED_WORKLIST)
+        assert_close(out.float().cpu().numpy(), ref, f"work list workspace {fill}")
+
+
+def test_work_list_schedule_refuses_multi_wave_grids():
+    d = dev(scaled(2))
+    p = pa.params_for(d, force_partitions=40, schedule=pa.PA_SCHED_WORKLIST)
+    rc, _ = pa.pa_plan(p, 16)
+    assert rc == pa.PA_ERR_UNSUPPORTED
+
+
+def test_work_list_full_size_long_context_sampled():
+    wl = config_workload(4, device="cuda:0")
+    out = pa.decode(wl, schedule=pa.PA_SCHED_WORKLIST)
+    torch.cuda.synchronize()
+    check_sampled(wl, out, sample_queries(wl, 32, seed=77), "work list long context")
