@@ -99,6 +99,25 @@ __device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long
   return v;
 }
 
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// epoch_touch split in two: `seen` is a value of the counter read earlier
+// (ld_relaxed_u64); a stale one is reset by a CAS that fails harmlessly if
+// another CTA of this call got there first.
+__device__ __forceinline__ void epoch_reset_if_stale(unsigned long long* c,
+                                                     unsigned long long seen,
+                                                     unsigned int epoch) {
+  if ((unsigned int)(seen >> 32) != epoch) atomicCAS(c, seen, (unsigned long long)epoch << 32);
+}
+
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 __device__ __forceinline__ void epoch_touch(unsigned long long* c, unsigned int epoch) {
   const unsigned long long cur = ld_acquire_u64(c);
   if ((unsigned int)(cur >> 32) != epoch) atomicCAS(c, cur, (unsigned long long)epoch << 32);

@@ -492,50 +492,106 @@ __device__ __forceinline__ void lse_merge(LseAcc& x, float m2, float z2, float4 
 // the work-list schedule, whose one-wave grid is launched cooperatively, so
 // every CTA of a unit is resident: each CTA publishes its partial (fence, then
 // an epoch-tagged arrival), waits until all nparts partials of its unit have
-// arrived, then merges a share of the unit's outputs -- one warp per (row,
-// 4 dims), its lanes striding over the partials with a running log-sum-exp
-// and a butterfly merge at the end.  Partials are read through L2 (ld.cg):
-// other SMs wrote them during this kernel.
+// arrived, then merges a share of the unit's outputs with a running
+// log-sum-exp: up to 32 partials, one warp per row with its lanes over the
+// dims; more, one CTA per (row, 16 dims) with its lanes over the partials in
+// 64-byte slices.  Partials are read through L2 (ld.cg): other SMs wrote
+// them during this kernel.
 // ---------------------------------------------------------------------------
 template <int D>
 __device__ __noinline__ void merge_unit_partials(const DecodeArgs& a, int b, int kvh, int part,
-                                                 int nparts, int row0, int Rs, int qoff) {
+                                                 int nparts, int row0, int Rs, int qoff,
+                                                 int touched) {
   __shared__ int s_go;
+  __shared__ float s_m[16], s_z[16];
+  __shared__ float4 s_o[16][4];
+  constexpr int C4 = D / 4;
+  constexpr int DC = 16;         // many partials: dims per (row, slice) item
+  constexpr int NSL = D / DC;    // slices per row
+  constexpr int LPP = DC / 4;    // lanes per partial's slice (one float4 each)
+  constexpr int PPW = 32 / LPP;  // partials per warp load
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nw = blockDim.x >> 5;
+  const bool few = nparts <= 32;
+  // Only CTAs with a share of the merge wait for the unit's arrivals; the
+  // rest publish their partial and leave (fewer pollers on the counter).
+  const bool share = few ? part * nw < Rs : part < Rs * NSL;
   __threadfence();
   __syncthreads();
   unsigned long long* cnt = a.done + (size_t)blockIdx.z * gridDim.y + blockIdx.y;
   if (threadIdx.x == 0) {
-    epoch_arrive(cnt, a.epoch);
-    s_go = epoch_wait(cnt, a.epoch, (unsigned)nparts);
+    if (!touched) epoch_touch(cnt, a.epoch);
+    atomicAdd(cnt, 1ull);
+    s_go = share && epoch_wait(cnt, a.epoch, (unsigned)nparts);
     __threadfence();
   }
   __syncthreads();
   if (!s_go) return;
-  constexpr int C4 = D / 4;
-  constexpr int BATCH = 4;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nw = blockDim.x >> 5;
   const size_t ubase = (size_t)(b * a.num_kv_heads + kvh) * a.max_parts;
-  for (int j = part * nw + warp; j < Rs * C4; j += nparts * nw) {
-    const int r = j / C4, c4 = j - (j / C4) * C4;
+  auto store = [&](int rr, int c4, const LseAcc& acc) {
+    const float inv = acc.z > 0.f ? 1.f / acc.z : 0.f;
+    const int i = rr / a.group, jj = rr - (rr / a.group) * a.group;
+    __nv_bfloat16* dp =
+        a.dst + ((size_t)(qoff + i) * a.num_q_heads + (size_t)kvh * a.group + jj) * D + c4 * 4;
+    *reinterpret_cast<__nv_bfloat162*>(dp) = __floats2bfloat162_rn(acc.o.x * inv, acc.o.y * inv);
+    *reinterpret_cast<__nv_bfloat162*>(dp + 2) = __floats2bfloat162_rn(acc.o.z * inv, acc.o.w * inv);
+  };
+  if (few) {
+    // Few partials: a warp per row, lanes over its dims (4 each), every
+    // partial's loads issued before the first merge.
+    constexpr int PB = 8;
+    for (int r = part * nw + warp; r < Rs; r += nparts * nw) {
+      const int rr = row0 + r;
+      for (int c4 = lane; c4 < C4; c4 += 32) {
+        LseAcc acc{kNegInf, 0.f, make_float4(0.f, 0.f, 0.f, 0.f)};
+        for (int p0 = 0; p0 < nparts; p0 += PB) {
+          float l[PB];
+          float4 o[PB];
+#pragma unroll
+          for (int u = 0; u < PB; ++u) {
+            const size_t base = (ubase + p0 + u) * a.max_rows + rr;
+            const bool in = p0 + u < nparts;
+            l[u] = in ? __ldcg(a.ws_lse + base) : kNegInf;
+            o[u] = in ? __ldcg(reinterpret_cast<const float4*>(a.ws_o + base * D) + c4)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int u = 0; u < PB; ++u) lse_merge(acc, l[u], 1.f, o[u]);
+        }
+        store(rr, c4, acc);
+      }
+    }
+    return;
+  }
+  // Many partials: a CTA per (row, 16-dim slice).  Its warps split the
+  // partials, LPP lanes reading one partial's slice (64 contiguous bytes), so
+  // a warp load covers PPW partials; lanes, then warps (through shared
+  // memory), merge with the same rescale.
+  const int sub = lane / LPP, c4 = lane - (lane / LPP) * LPP;
+  const size_t pst4 = (size_t)a.max_rows * D / 4;  // float4 stride between partials
+  const int step = nw * PPW;
+  constexpr int BATCH = 8;
+  for (int it = part; it < Rs * NSL; it += nparts) {
+    const int r = it / NSL, sl = it - (it / NSL) * NSL;
     const int rr = row0 + r;
+    const float* lse = a.ws_lse + ubase * a.max_rows + rr;
+    const float4* ob =
+        reinterpret_cast<const float4*>(a.ws_o + (ubase * a.max_rows + rr) * D + sl * DC) + c4;
     LseAcc acc{kNegInf, 0.f, make_float4(0.f, 0.f, 0.f, 0.f)};
-    for (int p0 = lane; p0 < nparts; p0 += 32 * BATCH) {
+    for (int p0 = warp * PPW + sub; p0 < nparts; p0 += BATCH * step) {
       float l[BATCH];
       float4 o[BATCH];
 #pragma unroll
       for (int u = 0; u < BATCH; ++u) {
-        const int p = p0 + 32 * u;
-        const size_t base = (ubase + p) * a.max_rows + rr;
-        l[u] = p < nparts ? __ldcg(a.ws_lse + base) : kNegInf;
-        o[u] = p < nparts ? __ldcg(reinterpret_cast<const float4*>(a.ws_o + base * D) + c4)
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
+        const int p = p0 + u * step;
+        l[u] = p < nparts ? __ldcg(lse + (size_t)p * a.max_rows) : kNegInf;
+        o[u] = p < nparts ? __ldcg(ob + (size_t)p * pst4) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
       for (int u = 0; u < BATCH; ++u) lse_merge(acc, l[u], 1.f, o[u]);
     }
 #pragma unroll
-    for (int off = 16; off; off >>= 1) {
+    for (int off = LPP; off < 32; off <<= 1) {
       const float m2 = __shfl_xor_sync(FULL, acc.m, off);
       const float z2 = __shfl_xor_sync(FULL, acc.z, off);
       float4 o2;
@@ -545,15 +601,20 @@ __device__ __noinline__ void merge_unit_partials(const DecodeArgs& a, int b, int
       o2.w = __shfl_xor_sync(FULL, acc.o.w, off);
       lse_merge(acc, m2, z2, o2);
     }
-    if (lane == 0) {
-      const float inv = acc.z > 0.f ? 1.f / acc.z : 0.f;
-      const int i = rr / a.group, jj = rr - (rr / a.group) * a.group;
-      __nv_bfloat16* dp =
-          a.dst + ((size_t)(qoff + i) * a.num_q_heads + (size_t)kvh * a.group + jj) * D + c4 * 4;
-      *reinterpret_cast<__nv_bfloat162*>(dp) = __floats2bfloat162_rn(acc.o.x * inv, acc.o.y * inv);
-      *reinterpret_cast<__nv_bfloat162*>(dp + 2) =
-          __floats2bfloat162_rn(acc.o.z * inv, acc.o.w * inv);
+    if (sub == 0) {
+      s_o[warp][c4] = acc.o;
+      if (c4 == 0) {
+        s_m[warp] = acc.m;
+        s_z[warp] = acc.z;
+      }
     }
+    __syncthreads();
+    if (warp == 0 && lane < LPP) {
+      LseAcc t{kNegInf, 0.f, make_float4(0.f, 0.f, 0.f, 0.f)};
+      for (int i = 0; i < nw; ++i) lse_merge(t, s_m[i], s_z[i], s_o[i][lane]);
+      store(rr, sl * LPP + lane, t);
+    }
+    __syncthreads();
   }
 }
 
@@ -586,11 +647,13 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
   __shared__ int s_qoff;
   __shared__ float s_fac[NCW][64], s_rowm[64], s_rowz[64];  // warp-merge factors (rows <= 64)
   __shared__ int s_c0[WL ? NSTAGE : 1];  // work list: each slot's first token; -1: stop
+  __shared__ int s_dtouch;                // work list: the arrival counter is this call's
 
   // Nothing here depends on the inputs: set up the pipeline while the
   // previous kernel on the stream may still be finishing (this kernel is
   // launched with programmatic stream serialization), then wait for it.
   if (threadIdx.x == 0) {
+    if constexpr (WL) s_dtouch = 0;
     prefetch_tensormap(&tmk);
     prefetch_tensormap(&tmv);
     for (int s = 0; s < NSTAGE; ++s) {
@@ -680,59 +743,67 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
     __syncwarp();
     const int nbox = TS / BR;
     const int nitem = nbox * 2;  // (box, K/V) per lane
-    unsigned long long* ctr = nullptr;
-    unsigned long long pend = 0;  // lane 0: the claim in flight (raw counter value)
-    int cur = 0, left = 0;        // claimed stages not yet issued: cur, cur+1, ...
-    if constexpr (WL) {
-      ctr = a.stage_ctr + (size_t)blockIdx.z * gridDim.y + blockIdx.y;
-      int first = 0;
-      if (lane == 0) {
-        epoch_touch(ctr, a.epoch);
-        first = claim_value(atomicAdd(ctr, (unsigned long long)NSTAGE), a.epoch);
-      }
-      cur = __shfl_sync(FULL, first, 0);
-      left = NSTAGE;
-    }
     const int nst_unit = (S - A + TS - 1) / TS;
-    int k = 0;
-    bool ok = true;
-    for (;; ++k) {
-      int c0;
-      int phys_w = -1;  // work list: this lane's box block, read for this stage
-      if constexpr (WL) {
-        if (left == 0) {
-          int v = 0;
-          if (lane == 0) v = claim_value(pend, a.epoch);
-          cur = __shfl_sync(FULL, v, 0);
-          left = 1;
-        }
-        const int st = cur++;
-        --left;
-        if (st >= nst_unit) break;
-        if (left == 0 && lane == 0) pend = atomicAdd(ctr, 1ull);
-        c0 = A + st * TS;
-        if (lane < nitem) {
-          const int bt0 = c0 + (lane >> 1) * BR;
-          if (bt0 < S && bt0 + BR > ulo) {
-            phys_w = a.block_tables[(size_t)b * a.max_blocks_per_seq + (bt0 >> a.block_shift)];
-            if (phys_w < 0 || phys_w >= a.num_blocks) {
-              atomicOr(&g_pa_status, PA_DEV_BAD_BLOCK);
-              phys_w = -1;
-            }
-          }
-        }
-      } else {
-        if (k >= nst) break;
-        c0 = p0 + k * TS;
+    // Work list: s_j is the j-th stage this CTA copies.  At iteration j the
+    // numbers of s_j .. s_j+2 are known (st_cur, st_n1, st_n2) and this lane's
+    // block-table entry for s_j was read at the end of iteration j - 2 into
+    // the register of j's parity (rawA / rawB); claims alternate between two
+    // in-flight atomics (pendA / pendB) the same way.  Values still in
+    // flight are never copied between registers, so no wait lands on an
+    // iteration earlier than the one that uses the value.
+    int st_cur = 0, st_n1 = 0, st_n2 = 0;
+    int rawA = 0, rawB = 0;
+    unsigned long long pendA = 0, pendB = 0;  // lane 0
+    int run = 0, run_left = 0;  // this CTA's fixed stages not yet taken: run, run + 1, ...
+    constexpr int kNoBox = INT_MIN;
+    // This lane's block-table entry for stage st (kNoBox: nothing to copy).
+    auto table_entry = [&](int st) -> int {
+      if (st >= nst_unit || lane >= nitem) return kNoBox;
+      const int bt0 = A + st * TS + (lane >> 1) * BR;
+      if (bt0 >= S || bt0 + BR <= ulo) return kNoBox;
+      return a.block_tables[(size_t)b * a.max_blocks_per_seq + (bt0 >> a.block_shift)];
+    };
+    constexpr int kFixed = NSTAGE + 2;  // work list: stages each CTA owns outright
+    unsigned long long seen_ctr = 0, seen_done = 0;  // lane 0: the counters as first read
+    unsigned long long* ctr = a.stage_ctr + (size_t)blockIdx.z * gridDim.y + blockIdx.y;
+    unsigned long long* done = a.done + (size_t)blockIdx.z * gridDim.y + blockIdx.y;
+    if constexpr (WL) {
+      // A ring's worth plus two stages per CTA are fixed (CTA `part` starts
+      // at stage part * kFixed), so the first copies wait for no claim; later
+      // stages come from the unit's counter, numbered past all the fixed
+      // ones.  The counters are read now and reset (if stale) after stage
+      // 0's copies; claims are resolved three stages ahead and block-table
+      // entries read two ahead, each waited for after a stage's copies are
+      // out, and the unit's block-table lines are prefetched into L2, spread
+      // over its CTAs.
+      if (lane == 0) {
+        seen_ctr = ld_relaxed_u64(ctr);
+        seen_done = ld_relaxed_u64(done);
       }
-      const int s = k % NSTAGE;
-      if (k >= NSTAGE) {
+      const int* tb = a.block_tables + (size_t)b * a.max_blocks_per_seq;
+      const int e1 = ((S - 1) >> a.block_shift) + 1;
+      for (int e = ((A >> a.block_shift) & ~31) + (part * 32 + lane) * 32; e < e1;
+           e += nparts * 32 * 32)
+        prefetch_l2(tb + e);
+      st_cur = min(part * kFixed, nst_unit);
+      st_n1 = min(st_cur + 1, nst_unit);
+      st_n2 = min(st_cur + 2, nst_unit);
+      run = st_cur + 3;
+      run_left = kFixed - 3;
+      rawA = table_entry(st_cur);
+      rawB = table_entry(st_n1);
+    }
+    const int dyn0 = nparts * kFixed;  // first stage handed out by the counter
+
+    // Copies stage number kk (ring slot kk % NSTAGE) of tokens [c0, c0 + TS);
+    // raw: the work list's block-table entry for this lane's box.  False if
+    // the wait for the slot timed out.
+    auto issue = [&](int kk, int c0, int raw) -> bool {
+      const int s = kk % NSTAGE;
+      if (kk >= NSTAGE) {
         bool got = true;
-        if (lane == 0) got = mbar_wait(smem_u32(&bars[NSTAGE + s]), ((k / NSTAGE) - 1) & 1);
-        if (!__shfl_sync(FULL, got, 0)) {
-          ok = false;
-          break;
-        }
+        if (lane == 0) got = mbar_wait(smem_u32(&bars[NSTAGE + s]), ((kk / NSTAGE) - 1) & 1);
+        if (!__shfl_sync(FULL, got, 0)) return false;
       }
       const int ta = max(c0, ulo), te = min(c0 + TS, p1);
       bool mine = false;
@@ -744,7 +815,16 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
         const int bt0 = c0 + j * BR;
         if (bt0 + BR > ta && bt0 < te) {
           const int jj = bt0 >> a.block_shift;
-          const int phys = WL ? phys_w : bt_s[jj - jb0];
+          int phys;
+          if constexpr (WL) {
+            phys = raw;
+            if (phys < 0 || phys >= a.num_blocks) {
+              atomicOr(&g_pa_status, PA_DEV_BAD_BLOCK);
+              phys = -1;
+            }
+          } else {
+            phys = bt_s[jj - jb0];
+          }
           if (phys >= 0) {
             mine = true;
             y = (phys * a.num_kv_heads + kvh) * a.block_size + (bt0 - (jj << a.block_shift));
@@ -762,6 +842,64 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
         tma_load_3d(smem_u32(smem) + dst, isv ? static_cast<const void*>(&tmv)
                                               : static_cast<const void*>(&tmk),
                     0, y, 0, smem_u32(&bars[s]));
+      return true;
+    };
+    // Work list, after stage kk's copies: the next stage numbers, the claim
+    // of kk's parity, and the block-table read for stage kk + 2 (same parity).
+    auto advance = [&](int kk, unsigned long long& pend, int& raw) {
+      if (kk == 0 && lane == 0) {  // open this CTA's claims
+        epoch_reset_if_stale(ctr, seen_ctr, a.epoch);
+        pendA = atomicAdd(ctr, 1ull);
+        pendB = atomicAdd(ctr, 1ull);
+        epoch_reset_if_stale(done, seen_done, a.epoch);
+        s_dtouch = 1;
+      }
+      int st_n3;
+      if (run_left > 0) {
+        st_n3 = min(run++, nst_unit);
+        --run_left;
+      } else {
+        int v = 0;
+        if (lane == 0) {
+          v = claim_value(pend, a.epoch);  // INT_MAX (stop) if not this call's
+          v = v >= nst_unit - dyn0 ? nst_unit : dyn0 + v;
+          pend = atomicAdd(ctr, 1ull);
+        }
+        st_n3 = __shfl_sync(FULL, v, 0);
+      }
+      st_cur = st_n1;
+      st_n1 = st_n2;
+      st_n2 = st_n3;
+      raw = table_entry(st_n1);
+    };
+
+    int k = 0;
+    bool ok = true;
+    if constexpr (!WL) {
+      for (; k < nst; ++k)
+        if (!issue(k, p0 + k * TS, 0)) {
+          ok = false;
+          break;
+        }
+    } else {
+      for (;; k += 2) {
+        if (st_cur >= nst_unit) break;
+        if (!issue(k, A + st_cur * TS, rawA)) {
+          ok = false;
+          break;
+        }
+        advance(k, pendA, rawA);
+        if (st_cur >= nst_unit) {
+          k += 1;
+          break;
+        }
+        if (!issue(k + 1, A + st_cur * TS, rawB)) {
+          k += 1;
+          ok = false;
+          break;
+        }
+        advance(k + 1, pendB, rawB);
+      }
     }
     const int issued = k;
     if (WL && ok && lane == 0) {
@@ -1124,7 +1262,7 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
     }
   }
   if constexpr (WL)
-    if (nparts > 1) merge_unit_partials<D>(a, b, kvh, part, nparts, row0, Rs, qoff);
+    if (nparts > 1) merge_unit_partials<D>(a, b, kvh, part, nparts, row0, Rs, qoff, s_dtouch);
 }
 
 // ---------------------------------------------------------------------------
