@@ -246,7 +246,14 @@ int pa_unreachable_blocks(int32_t *count, const int32_t *seqLens, const int32_t 
  * seqLens, queryLens (and windows) from host memory into the caller's
  * workspace, runs pa_decode, copies dst back, and synchronises the stream.
  * The KV caches stay on the device (they are resident state).  Host buffers
- * should be pinned for asynchronous copies.
+ * should be pinned: a pinned buffer that is mapped into the current context
+ * (CUDA's default for pinned memory under unified addressing) is read in
+ * place by one staging kernel for all inputs, and a mapped, 16-byte aligned
+ * dst_host is written in place by the kernels, so no copy engine is used
+ * for it; other (pageable, unmapped) buffers are moved with
+ * cudaMemcpyAsync.  The library checks with the driver that each buffer
+ * lies inside one pinned allocation before reading or writing it in place.
+ * All host buffers must stay valid and unmodified until the call returns.
  *   dst_host          host bf16 [sum(queryLens)][H_q][head_dim]
  *   q_host            host bf16 or FP8 codes (q_dtype), same shape
  *   blockTables_host, seqLens_host, queryLens_host  host int32

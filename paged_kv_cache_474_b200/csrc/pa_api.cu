@@ -53,6 +53,7 @@ constexpr int TS = pa::kStageTokens;
 constexpr int kMinPartTokens = 256;
 constexpr int kManyUnitsMinTokens = 2048;
 constexpr int kManyUnitsMaxTokens = 4096;
+constexpr unsigned long long kStageMaxBlocks = 512;  // CTAs per staging copy (256 threads each)
 
 bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
@@ -325,6 +326,49 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
       fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
   });
   return fn;
+}
+
+// The device address of a host buffer that kernels may read and write in
+// place: pinned, mapped into the current context at the same address, with
+// [p, p + bytes) inside one allocation.  nullptr for anything else (pageable
+// or device memory, a range running past its allocation, a driver without the
+// query), which the caller then moves with cudaMemcpyAsync.
+void* mapped_host(const void* p, size_t bytes) {
+  static PFN_cuPointerGetAttributes_v7000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuPointerGetAttributes", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuPointerGetAttributes_v7000>(f);
+  });
+  if (!fn || !p || bytes == 0) return nullptr;
+  CUpointer_attribute at[5] = {CU_POINTER_ATTRIBUTE_MEMORY_TYPE, CU_POINTER_ATTRIBUTE_DEVICE_POINTER,
+                               CU_POINTER_ATTRIBUTE_RANGE_START_ADDR,
+                               CU_POINTER_ATTRIBUTE_RANGE_SIZE, CU_POINTER_ATTRIBUTE_MAPPED};
+  // every slot is 8 bytes and zeroed: the driver writes 1 to 8 of them
+  unsigned long long mtype = 0, dptr = 0, start = 0, size = 0, mapped = 0;
+  void* data[5] = {&mtype, &dptr, &start, &size, &mapped};
+  const CUdeviceptr addr = (CUdeviceptr)reinterpret_cast<uintptr_t>(p);
+  if (fn(5, at, data, addr) != CUDA_SUCCESS) return nullptr;
+  if ((unsigned int)mtype != CU_MEMORYTYPE_HOST || (mapped & 0xffu) == 0 || dptr != addr)
+    return nullptr;
+  if (addr < start || addr - start > size || bytes > size - (addr - start)) return nullptr;
+  return reinterpret_cast<void*>(static_cast<uintptr_t>(dptr));
+}
+
+// One staging copy: the widest piece both addresses and the size allow.
+pa::StageCopy stage_copy(const void* src, void* dst, size_t bytes) {
+  const uintptr_t m = reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst) | bytes;
+  pa::StageCopy c;
+  c.src = src;
+  c.dst = dst;
+  c.unit = (m & 15u) == 0 ? 16 : (m & 3u) == 0 ? 4 : 1;
+  c.units = bytes / c.unit;
+  c.first_block = 0;
+  return c;
 }
 
 // 3-D map of a KV cache viewed as (box width W bytes, rows, row bytes / W
@@ -666,14 +710,38 @@ int pa_decode_host(void* dst_host, const void* q_host, const void* kCache, const
   char* d_W = d_L + align256((size_t)B * 4);
   char* d_split = d_W + align256((size_t)B * 4);
 
+  // Inputs in.  Pinned host buffers that are mapped into this context are
+  // read in place by one staging kernel (a DMA copy per buffer costs several
+  // microseconds of fixed latency each); the others are copied.
+  struct In {
+    const void* src;
+    void* dst;
+    size_t bytes;
+  } ins[5] = {{q_host, d_q, qbytes_raw},
+              {blockTables_host, d_bt, btbytes},
+              {seqLens_host, d_S, (size_t)B * 4},
+              {queryLens_host, d_L, (size_t)B * 4},
+              {params->windows, d_W, params->windows ? (size_t)B * 4 : 0}};
+  pa::StageArgs sa;
+  memset(&sa, 0, sizeof sa);
   cudaError_t e = cudaSuccess;
-  if (qbytes_raw) e = cudaMemcpyAsync(d_q, q_host, qbytes_raw, cudaMemcpyHostToDevice, st);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(d_bt, blockTables_host, btbytes, cudaMemcpyHostToDevice, st);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(d_S, seqLens_host, (size_t)B * 4, cudaMemcpyHostToDevice, st);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(d_L, queryLens_host, (size_t)B * 4, cudaMemcpyHostToDevice, st);
-  if (e == cudaSuccess && params->windows)
-    e = cudaMemcpyAsync(d_W, params->windows, (size_t)B * 4, cudaMemcpyHostToDevice, st);
+  for (const In& in : ins) {
+    if (!in.bytes) continue;
+    const void* mapped = mapped_host(in.src, in.bytes);
+    if (mapped) {
+      pa::StageCopy c = stage_copy(mapped, in.dst, in.bytes);
+      c.first_block = sa.blocks;
+      sa.blocks += (int)std::min<unsigned long long>((c.units + 255) / 256, kStageMaxBlocks);
+      sa.c[sa.n++] = c;
+    } else if (e == cudaSuccess) {
+      e = cudaMemcpyAsync(in.dst, in.src, in.bytes, cudaMemcpyHostToDevice, st);
+    }
+  }
+  if (e == cudaSuccess && sa.n) e = pa::launch_stage(sa, st);
   if (e != cudaSuccess) return fail(PA_ERR_CUDA, "host-to-device copy: %s", cudaGetErrorString(e));
+  // Output: a mapped, 16-byte aligned dst is written by the kernels in place.
+  void* dst_mapped = aligned16(dst_host) ? mapped_host(dst_host, dbytes_raw) : nullptr;
+  if (dst_mapped) d_dst = static_cast<char*>(dst_mapped);
 
   if (qlen > 0) {
     pa_params dp = *params;
@@ -687,7 +755,8 @@ int pa_decode_host(void* dst_host, const void* q_host, const void* kCache, const
                      scale, window, kvBlockSize, &dp, st, span, qlen);
     if (rc) return rc;
   }
-  if (dbytes_raw) e = cudaMemcpyAsync(dst_host, d_dst, dbytes_raw, cudaMemcpyDeviceToHost, st);
+  if (dbytes_raw && !dst_mapped)
+    e = cudaMemcpyAsync(dst_host, d_dst, dbytes_raw, cudaMemcpyDeviceToHost, st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return fail(PA_ERR_CUDA, "device-to-host copy: %s", cudaGetErrorString(e));
   return succeed();

@@ -533,8 +533,8 @@ __device__ __noinline__ void merge_unit_partials(const DecodeArgs& a, int b, int
     const int i = rr / a.group, jj = rr - (rr / a.group) * a.group;
     __nv_bfloat16* dp =
         a.dst + ((size_t)(qoff + i) * a.num_q_heads + (size_t)kvh * a.group + jj) * D + c4 * 4;
-    *reinterpret_cast<__nv_bfloat162*>(dp) = __floats2bfloat162_rn(acc.o.x * inv, acc.o.y * inv);
-    *reinterpret_cast<__nv_bfloat162*>(dp + 2) = __floats2bfloat162_rn(acc.o.z * inv, acc.o.w * inv);
+    *reinterpret_cast<uint2*>(dp) = make_uint2(pack_bf16x2(acc.o.x * inv, acc.o.y * inv),
+                                               pack_bf16x2(acc.o.z * inv, acc.o.w * inv));
   };
   if (few) {
     // Few partials: a warp per row, lanes over its dims (4 each), every
@@ -1250,8 +1250,9 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
       const int i = rr / a.group, j = rr - (rr / a.group) * a.group;
       __nv_bfloat16* dp =
           a.dst + ((size_t)(qoff + i) * a.num_q_heads + (size_t)kvh * a.group + j) * D + c4 * 4;
-      *reinterpret_cast<__nv_bfloat162*>(dp) = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-      *reinterpret_cast<__nv_bfloat162*>(dp + 2) = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+      // one 8-byte store per lane: a warp writes whole 32-byte sectors
+      *reinterpret_cast<uint2*>(dp) = make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv),
+                                                 pack_bf16x2(acc.z * inv, acc.w * inv));
     } else {
       const float inv = Z > 0.f ? a.v_scale / Z : 0.f;
       const size_t base =
@@ -1360,8 +1361,10 @@ __global__ void __launch_bounds__(512) pa_reduce_kernel(const __grid_constant__ 
     __nv_bfloat16* dp = a.dst +
                         ((size_t)(s_qoff + i) * a.num_q_heads + (size_t)kvh * a.group + j) * D +
                         ch * DC + lane * 4;
-    *reinterpret_cast<__nv_bfloat162*>(dp) = __floats2bfloat162_rn(t.o.x * inv, t.o.y * inv);
-    *reinterpret_cast<__nv_bfloat162*>(dp + 2) = __floats2bfloat162_rn(t.o.z * inv, t.o.w * inv);
+    // one 8-byte store per lane: a warp writes whole 32-byte sectors (and
+    // whole write requests when dst is mapped host memory)
+    *reinterpret_cast<uint2*>(dp) = make_uint2(pack_bf16x2(t.o.x * inv, t.o.y * inv),
+                                               pack_bf16x2(t.o.z * inv, t.o.w * inv));
   }
 }
 
@@ -1423,6 +1426,53 @@ __global__ void __launch_bounds__(1024) pa_ranges_kernel(int32_t* lo, int32_t* h
     __syncthreads();
     if (tid == blockDim.x - 1) carry = off + L;
     __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Staging copies of the host-buffer entry point.  Each copy owns a run of
+// CTAs; a thread issues up to four loads before its stores, so a CTA keeps
+// 256 x 4 pieces in flight across the host link.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) pa_stage_kernel(const __grid_constant__ StageArgs s) {
+  // The partition kernel may launch now: it waits on griddepcontrol for this
+  // grid's completion (and its writes) before reading any input.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  int c = 0;
+  while (c + 1 < s.n && (int)blockIdx.x >= s.c[c + 1].first_block) ++c;
+  const StageCopy& sc = s.c[c];
+  const int nb = (c + 1 < s.n ? s.c[c + 1].first_block : s.blocks) - sc.first_block;
+  const unsigned long long stride = (unsigned long long)nb * blockDim.x;
+  const unsigned long long t =
+      (unsigned long long)(blockIdx.x - sc.first_block) * blockDim.x + threadIdx.x;
+  if (sc.unit == 16) {
+    const uint4* src = static_cast<const uint4*>(sc.src);
+    uint4* dst = static_cast<uint4*>(sc.dst);
+    for (unsigned long long u = t; u < sc.units; u += 4 * stride) {
+      uint4 v[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (u + j * stride < sc.units) v[j] = src[u + j * stride];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (u + j * stride < sc.units) dst[u + j * stride] = v[j];
+    }
+  } else if (sc.unit == 4) {
+    const uint32_t* src = static_cast<const uint32_t*>(sc.src);
+    uint32_t* dst = static_cast<uint32_t*>(sc.dst);
+    for (unsigned long long u = t; u < sc.units; u += 4 * stride) {
+      uint32_t v[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (u + j * stride < sc.units) v[j] = src[u + j * stride];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (u + j * stride < sc.units) dst[u + j * stride] = v[j];
+    }
+  } else {
+    const uint8_t* src = static_cast<const uint8_t*>(sc.src);
+    uint8_t* dst = static_cast<uint8_t*>(sc.dst);
+    for (unsigned long long u = t; u < sc.units; u += stride) dst[u] = src[u];
   }
 }
 
@@ -1703,6 +1753,12 @@ cudaError_t launch_unreachable(int32_t* count, const int32_t* seq_lens, const in
                                cudaStream_t stream) {
   pa_unreachable_kernel<<<(batch + 255) / 256, 256, 0, stream>>>(count, seq_lens, query_lens, window,
                                                                   windows, block_shift, batch);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_stage(const StageArgs& s, cudaStream_t stream) {
+  if (s.n <= 0 || s.n > kMaxStageCopies || s.blocks <= 0) return cudaErrorInvalidValue;
+  pa_stage_kernel<<<s.blocks, 256, 0, stream>>>(s);
   return cudaGetLastError();
 }
 

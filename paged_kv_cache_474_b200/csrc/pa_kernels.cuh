@@ -105,6 +105,27 @@ cudaError_t launch_unreachable(int32_t* count, const int32_t* seq_lens, const in
                                int window, const int32_t* windows, int block_shift, int batch,
                                cudaStream_t stream);
 
+// Staging copies for the host-buffer entry point: up to kMaxStageCopies
+// buffers copied by one kernel (one launch instead of one DMA copy per
+// buffer).  Sources are device addresses of pinned, mapped host buffers.
+constexpr int kMaxStageCopies = 6;
+struct StageCopy {
+  const void* src;
+  void* dst;
+  unsigned long long units;  // number of `unit`-byte pieces
+  int unit;                  // 16, 4 or 1: the widest both addresses and the size allow
+  int first_block;           // the copy's CTAs are [first_block, next copy's first_block)
+};
+struct StageArgs {
+  StageCopy c[kMaxStageCopies];
+  int n;
+  int blocks;  // grid size
+};
+
+// Launches the staging copies; the next kernel on the stream may be launched
+// while they run (it waits for their completion before reading anything).
+cudaError_t launch_stage(const StageArgs& s, cudaStream_t stream);
+
 // Reads (and optionally clears) the device status word.
 cudaError_t read_status(unsigned int* status, bool clear, cudaStream_t stream);
 

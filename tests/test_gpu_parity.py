@@ -206,30 +206,66 @@ def test_visible_ranges_match_oracle_exactly():
         assert np.array_equal(hi.cpu().numpy(), rhi)
 
 
-def test_host_entry_point_matches_device_path():
-    wl = scaled(5)
+def _host_buffer(arr, kind, offset=0):
+    """A host copy of ``arr`` (a CPU tensor): pinned (read in place by the
+    library's staging kernel) or pageable (copied), optionally starting
+    ``offset`` bytes into a larger buffer of the same kind."""
+    raw = arr.contiguous().view(torch.uint8).reshape(-1)
+    buf = torch.zeros(raw.numel() + offset + 16, dtype=torch.uint8)
+    if kind == "pinned":
+        buf = buf.pin_memory()
+    buf[offset:offset + raw.numel()] = raw
+    return buf, buf.data_ptr() + offset
+
+
+# kinds of q / tables+lengths+windows / dst host buffers, and byte offsets of
+# q, tables and dst inside their buffers (offsets that break 16-byte or 4-byte
+# alignment take the narrower staging copies or the copy-back path)
+HOST_CASES = {
+    "pinned": (("pinned", "pinned", "pinned"), (0, 0, 0)),
+    "pageable": (("pageable", "pageable", "pageable"), (0, 0, 0)),
+    "mixed": (("pinned", "pageable", "pinned"), (0, 0, 0)),
+    "offsets": (("pinned", "pinned", "pinned"), (2, 4, 2)),
+    "offsets16": (("pinned", "pinned", "pinned"), (16, 32, 48)),
+}
+
+
+@pytest.mark.parametrize("case", list(HOST_CASES))
+@pytest.mark.parametrize("cfg", [2, 5])
+def test_host_entry_point_matches_device_path(cfg, case):
+    (kq, kt, kd), (oq, ot, od) = HOST_CASES[case]
+    wl = scaled(cfg)
     d = dev(wl)
     ref = pa.decode(d)
-    s, l, w = wl.host_lists()
     p = pa.make_params(batch=wl.batch, num_q_heads=wl.num_q_heads,
                        num_kv_heads=wl.num_kv_heads, head_dim=wl.head_dim,
                        num_blocks=wl.num_blocks, max_blocks_per_seq=wl.max_blocks_per_seq)
-    S = wl.seq_lens.numpy().copy()
-    L = wl.query_lens.numpy().copy()
-    W = wl.windows.numpy().copy()
-    p.windows = W.ctypes.data
-    n = pa.pa_host_workspace_size(p, wl.block_size, wl.window, S.ctypes.data, L.ctypes.data)
+    keep = []
+
+    def host(t, kind, off=0):
+        buf, ptr = _host_buffer(t, kind, off)
+        keep.append(buf)
+        return ptr
+    S = host(wl.seq_lens, kt)
+    L = host(wl.query_lens, kt)
+    if wl.windows is not None:
+        p.windows = host(wl.windows, kt)
+    n = pa.pa_host_workspace_size(p, wl.block_size, wl.window, S, L)
     ws = torch.empty(n, dtype=torch.uint8, device="cuda:0")
     p.workspace, p.workspace_bytes = ws.data_ptr(), n
-    q_host = wl.q.contiguous().pin_memory()
-    out_host = torch.empty_like(wl.q).pin_memory()
-    bt = wl.block_tables.contiguous().numpy()
-    rc = pa.pa_decode_host(out_host.data_ptr(), q_host.data_ptr(), d.k_cache.data_ptr(),
-                           d.v_cache.data_ptr(), bt.ctypes.data, S.ctypes.data, L.ctypes.data,
-                           wl.scale, wl.window, wl.block_size, p,
-                           pa._stream_handle())
-    assert rc == pa.PA_OK, pa.pa_last_error()
-    assert torch.equal(out_host, ref.cpu())
+    q = host(wl.q, kq, oq)
+    bt = host(wl.block_tables, kt, ot)
+    out_buf, out_ptr = _host_buffer(torch.full(wl.q.shape, float("nan"), dtype=torch.bfloat16),
+                                    kd, od)
+    for _ in range(2):   # twice: the second call overwrites the first's output in place
+        rc = pa.pa_decode_host(out_ptr, q, d.k_cache.data_ptr(), d.v_cache.data_ptr(), bt, S, L,
+                               wl.scale, wl.window, wl.block_size, p, pa._stream_handle())
+        assert rc == pa.PA_OK, pa.pa_last_error()
+        nbytes = ref.numel() * 2
+        got = out_buf[od:od + nbytes].view(torch.bfloat16).reshape(ref.shape)
+        assert torch.equal(got, ref.cpu())
+    # bytes around dst are untouched
+    assert torch.all(out_buf[:od] == 0) and torch.all(out_buf[od + nbytes:] == 0)
 
 
 # ---------------------------------------------------- full size, sampled
