@@ -1277,12 +1277,15 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
 // share a partial and a warp reads 32/LPP partials per load; each lane loads
 // lse_p with its O_p slice (BATCH partials in flight) and keeps a running
 // (max, sum, weighted sum), merged across the lanes of a slice and then
-// across warps with the same rescale.  Only the lengths are read before the
-// partials, so a row costs two dependent trips to L2.  Rows with hundreds of
-// partials split head_dim over several CTAs so more SMs pull partials from
-// L2.  Launched with programmatic stream serialization: it may be scheduled
-// while the partition kernel drains and waits on griddepcontrol before
-// reading.
+// across warps with the same rescale.  Rows with hundreds of partials split
+// head_dim over several CTAs so more SMs pull partials from L2.  Launched
+// with programmatic stream serialization: it is scheduled while the partition
+// kernel drains.  The lengths, windows and the row's q offset are read before
+// griddepcontrol.wait: they are inputs of the call, which the partition
+// kernel reads too, and it triggers this launch only after its own
+// griddepcontrol.wait, so whatever wrote them has completed.  Only the
+// partials are read after the wait: one trip to L2 once the partition grid
+// is done.
 // ---------------------------------------------------------------------------
 template <int D, int DSPLIT>
 __global__ void __launch_bounds__(512) pa_reduce_kernel(const __grid_constant__ DecodeArgs a) {
@@ -1294,7 +1297,6 @@ __global__ void __launch_bounds__(512) pa_reduce_kernel(const __grid_constant__ 
   __shared__ float4 s_o[16][LPP];
   __shared__ int s_qoff;
 
-  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int rr = blockIdx.x / DSPLIT, ch = blockIdx.x - (blockIdx.x / DSPLIT) * DSPLIT;
   const int kvh = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -1312,6 +1314,7 @@ __global__ void __launch_bounds__(512) pa_reduce_kernel(const __grid_constant__ 
   const int A = union_lo(S, L, w) & ~(kStageTokens - 1);
   const int nparts = (S - A + a.part_tokens - 1) / a.part_tokens;
   if (nparts <= 1 || nparts > a.max_parts) return;
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the partials are complete
 
   const int sub = lane / LPP, c4 = lane - (lane / LPP) * LPP;
   const size_t ubase = (size_t)(b * a.num_kv_heads + kvh) * a.max_parts;
