@@ -430,6 +430,11 @@ __global__ void __launch_bounds__(32 * (NCW + 1), (NCW <= 4 ? 2 : 1))
 // tile is dim 2g and row g+8 is dim 2g+1.  q_scale * k_scale is folded into
 // the score scale and v_scale into the output normalisation.
 // ---------------------------------------------------------------------------
+// Lazy running maximum of the tensor-core kernel's online softmax (log2
+// units): 2^8 = 256 bounds the unnormalised probabilities, far inside the
+// range of the bf16 and f16 P operands.
+constexpr float kLazyMax = 8.f;
+
 template <int D, bool F8>
 struct MmaTraits {
   static constexpr int ROW_BYTES = F8 ? D : 2 * D;                  // one token of one kv head
@@ -1078,10 +1083,14 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
             mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 4));
             mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 8));
             mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 16));
-            const float mn = fmaxf(m_r[n][j], mx);
+            // The running maximum moves only when the chunk's maximum passes it
+            // by more than kLazyMax (log2 units): probabilities stay below
+            // 2^kLazyMax, and after the first chunks O is rarely rescaled.
+            const bool up = mx > m_r[n][j] + kLazyMax;  // m_r = -inf: any finite mx
+            const float mn = up ? mx : m_r[n][j];
             const float mu = (mn == kNegInf) ? 0.f : mn;
-            al[n][j] = (mn == kNegInf) ? 1.f : ex2(m_r[n][j] - mu);
-            any_rescale |= (al[n][j] != 1.f);
+            al[n][j] = up ? ex2(m_r[n][j] - mu) : 1.f;  // first update: 2^-inf = 0 (O, l are 0)
+            any_rescale |= up;
             m_r[n][j] = mn;
             p[n][j] = ex2(v[j] - mu);
             p[n][j + 2] = ex2(v[j + 2] - mu);
