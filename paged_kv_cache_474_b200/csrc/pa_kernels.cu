@@ -455,17 +455,30 @@ struct MmaCombine {
   static constexpr int BYTES = (ACC_FLOATS + L_FLOATS + M_FLOATS) * 4;
 };
 
-// Byte offset, within a box, of 16-byte chunk `chunk` of row lt (lt < 16,
-// relative to a 16-row aligned chunk start).  128-byte box rows: half
-// (chunk / 8) of the box, row lt, chunk position swizzled by the row's low
-// three bits.  64-byte box rows (FP8, head_dim 64; 64-byte swizzle): chunk
-// position swizzled by bits 1..2 of the row.
+// Byte offset, within a box, of 16-byte chunk c = 2k + ck (ck in {0, 1}) of
+// row lt (lt < 16, relative to a 16-row aligned chunk start).  128-byte box
+// rows: half (c / 8) of the box (each half BR * 128 bytes), row lt, chunk
+// position (c & 7) ^ (lt & 7) (the 128-byte swizzle); 64-byte rows (FP8,
+// head_dim 64; 64-byte swizzle): chunk position (c & 3) ^ ((lt >> 1) & 3).
+// 2k only touches chunk bits 1..3 and ck only bit 0, so the offset splits into
+// a per-lane part, box_lane_off(lt, ck), computed once per warp, and a
+// per-step part that is one XOR with a constant (and, for the second half,
+// one add) once k is unrolled: (k >> 2) * half + (lane ^ (((2k) & 7) << 4)),
+// or lane ^ (((2k) & 3) << 4) for 64-byte rows.
 template <int BOXW>
-__device__ __forceinline__ uint32_t box_off(int lt, int chunk, int BR) {
+__device__ __forceinline__ uint32_t box_lane_off(int lt, int ck) {
   if constexpr (BOXW == 128)
-    return (uint32_t)((chunk >> 3) * BR * 128 + lt * 128 + (((chunk & 7) ^ (lt & 7)) << 4));
+    return (uint32_t)(lt * 128 + ((ck ^ (lt & 7)) << 4));
   else
-    return (uint32_t)(lt * 64 + (((chunk & 3) ^ ((lt >> 1) & 3)) << 4));
+    return (uint32_t)(lt * 64 + ((ck ^ ((lt >> 1) & 3)) << 4));
+}
+
+template <int BOXW>
+__device__ __forceinline__ uint32_t box_step_off(int k, uint32_t lane_off, uint32_t half) {
+  if constexpr (BOXW == 128)
+    return (uint32_t)(k >> 2) * half + (lane_off ^ (uint32_t)(((2 * k) & 7) << 4));
+  else
+    return lane_off ^ (uint32_t)(((2 * k) & 3) << 4);
 }
 
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
@@ -938,6 +951,9 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
     // (FP8 V uses the K addresses: its x4 covers tokens 0-7 / 8-15 of two chunks.)
     const int lt_v = F8 ? lt_k : ((lane >> 4) << 3) + (lane & 7);
     const int ck_v = F8 ? ck_k : (lane >> 3) & 1;
+    const uint32_t kofs = box_lane_off<T::BOXW>(lt_k, ck_k);
+    const uint32_t vofs = box_lane_off<T::BOXW>(lt_v, ck_v);
+    const uint32_t half = (uint32_t)BR * 128u;
     int lo_max, hi_min, dummy;
     query_range(S, L, L - 1, w, lo_max, dummy);  // the last token sees the latest start
     query_range(S, L, 0, w, dummy, hi_min);      // the first token sees the earliest end
@@ -1038,7 +1054,7 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
 #pragma unroll
           for (int kp = 0; kp < T::KSTEPS / 2; ++kp) {
             uint32_t r[4];
-            ldsm_x4(Ks + cbase + box_off<T::BOXW>(lt_k, kp * 2 + ck_k, BR), r[0], r[1], r[2], r[3]);
+            ldsm_x4(Ks + cbase + box_step_off<T::BOXW>(kp, kofs, half), r[0], r[1], r[2], r[3]);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               uint32_t ka[4];
@@ -1054,7 +1070,7 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
 #pragma unroll
           for (int ks = 0; ks < T::KSTEPS; ++ks) {
             uint32_t ka[4];
-            ldsm_x4(Ks + cbase + box_off<T::BOXW>(lt_k, ks * 2 + ck_k, BR), ka[0], ka[1], ka[2],
+            ldsm_x4(Ks + cbase + box_step_off<T::BOXW>(ks, kofs, half), ka[0], ka[1], ka[2],
                     ka[3]);
 #pragma unroll
             for (int n = 0; n < N8; ++n)
@@ -1138,7 +1154,7 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
 #pragma unroll
             for (int mp = 0; mp < T::MD / 2; ++mp) {
               uint32_t r[4];
-              ldsm_x4_t(Vs + cbase + box_off<T::BOXW>(lt_v, mp * 2 + ck_v, BR), r[0], r[1], r[2],
+              ldsm_x4_t(Vs + cbase + box_step_off<T::BOXW>(mp, vofs, half), r[0], r[1], r[2],
                         r[3]);
 #pragma unroll
               for (int h = 0; h < 2; ++h) {
@@ -1160,7 +1176,7 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
 #pragma unroll
             for (int md = 0; md < T::MD; ++md) {
               uint32_t va[4];
-              ldsm_x4_t(Vs + cbase + box_off<T::BOXW>(lt_v, md * 2 + ck_v, BR), va[0], va[1],
+              ldsm_x4_t(Vs + cbase + box_step_off<T::BOXW>(md, vofs, half), va[0], va[1],
                         va[2], va[3]);
               if constexpr (MK) {
                 va[0] &= mk_lo;
