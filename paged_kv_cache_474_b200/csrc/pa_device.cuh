@@ -161,6 +161,16 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
       : "memory");
 }
 
+// The same bulk copy with an L2 cache policy (createpolicy).
+__device__ __forceinline__ void bulk_g2s_hint(uint32_t dst, const void* src, uint32_t bytes,
+                                              uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1], %2, [%3], %4;" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar), "l"(policy)
+      : "memory");
+}
+
 // 2-D tiled TMA load global -> shared (no multicast) of the box at (x, y)
 // of `map` (a __grid_constant__ kernel parameter); completes the box's bytes
 // on `bar`.  x * element size must be a multiple of 16 bytes.
@@ -181,6 +191,25 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* map, int x
       " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
       : "memory");
+}
+
+// The same load with an L2 cache policy (createpolicy), e.g. evict-first for
+// data that is read once.
+__device__ __forceinline__ void tma_load_3d_hint(uint32_t dst, const void* map, int x, int y,
+                                                 int z, uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar), "l"(policy)
+      : "memory");
+}
+
+// L2 policy whose lines are evicted first: the KV stream, read once, then
+// leaves block tables, lengths, q and partials in L2.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
 }
 
 __device__ __forceinline__ void prefetch_tensormap(const void* map) {

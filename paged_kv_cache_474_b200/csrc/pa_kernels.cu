@@ -154,6 +154,7 @@ __global__ void __launch_bounds__(32 * (NCW + 1), (NCW <= 4 ? 2 : 1))
 
   if (warp == 0) {
     // ------------------------------ copy warp ------------------------------
+    const uint64_t kv_policy = l2_evict_first_policy();  // K/V rows are read once
     bool ok = true;
     int issued = 0;
     for (int k = 0; k < nst; ++k) {
@@ -188,7 +189,8 @@ __global__ void __launch_bounds__(32 * (NCW + 1), (NCW <= 4 ? 2 : 1))
       const uint32_t total = __reduce_add_sync(FULL, my_bytes);
       if (lane == 0) mbar_arrive_expect_tx(smem_u32(&bars[s]), total);
       __syncwarp();
-      if (my_bytes) bulk_g2s(smem_u32(smem) + dsto, src, my_bytes, smem_u32(&bars[s]));
+      if (my_bytes)
+        bulk_g2s_hint(smem_u32(smem) + dsto, src, my_bytes, smem_u32(&bars[s]), kv_policy);
       issued = k + 1;
     }
     // Drain: make sure no copy this warp issued is still in flight.
@@ -813,6 +815,7 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
     }
     const int dyn0 = nparts * kFixed;  // first stage handed out by the counter
 
+    const uint64_t kv_policy = l2_evict_first_policy();  // K/V are read once
     // Copies stage number kk (ring slot kk % NSTAGE) of tokens [c0, c0 + TS);
     // raw: the work list's block-table entry for this lane's box.  False if
     // the wait for the slot timed out.
@@ -857,9 +860,9 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
       }
       __syncwarp();
       if (mine)
-        tma_load_3d(smem_u32(smem) + dst, isv ? static_cast<const void*>(&tmv)
-                                              : static_cast<const void*>(&tmk),
-                    0, y, 0, smem_u32(&bars[s]));
+        tma_load_3d_hint(smem_u32(smem) + dst,
+                         isv ? static_cast<const void*>(&tmv) : static_cast<const void*>(&tmk), 0,
+                         y, 0, smem_u32(&bars[s]), kv_policy);
       return true;
     };
     // Work list, after stage kk's copies: the next stage numbers, the claim

@@ -348,6 +348,7 @@ __global__ void __maxnreg__(80)
     __syncwarp();
     const int nbox = kTcStage / BR;
     const int nitem = nbox * 2;  // (box, K/V) per lane: at most 16
+    const uint64_t kv_policy = l2_evict_first_policy();  // K/V codes are read once
     int k = 0;
     for (; k < nst; ++k) {
       const int s = k % NS;
@@ -385,9 +386,9 @@ __global__ void __maxnreg__(80)
       }
       __syncwarp();
       if (mine)
-        tma_load_3d(smem_u32(smem) + dst, isv ? static_cast<const void*>(&tmv)
-                                              : static_cast<const void*>(&tmk),
-                    0, y, 0, smem_u32(&full[s]));
+        tma_load_3d_hint(smem_u32(smem) + dst,
+                         isv ? static_cast<const void*>(&tmv) : static_cast<const void*>(&tmk), 0,
+                         y, 0, smem_u32(&full[s]), kv_policy);
     }
     const int issued = k;
     if (ok && lane == 0) {
