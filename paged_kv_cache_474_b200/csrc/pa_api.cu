@@ -527,6 +527,13 @@ int decode_impl(void* dst, const void* q, const void* kCache, const void* vCache
   a.num_slabs = in.grid_y / p->num_kv_heads;
 
   const dim3 grid(in.grid_x, in.grid_y, in.grid_z);
+  // One wave of window-free partitions (the few-units plan): a CTA's first
+  // copies need not wait for the lengths.  With many ragged rows (several
+  // waves) the copies for empty partitions would cost more than they save.
+  a.spec_first_stage = in.variant == PA_VARIANT_MMA && !in.worklist && !p->windows &&
+                       window == 0 &&
+                       (long long)in.grid_x * in.grid_y * in.grid_z <=
+                           (long long)in.num_sms * in.ctas_per_sm;
   cudaEvent_t ev0 = nullptr, ev1 = nullptr;
   if (p->profile_events) {
     ev0 = static_cast<cudaEvent_t>(p->profile_events[0]);

@@ -691,16 +691,55 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
   // can fetch the partition's block-table slice while the lengths are still
   // in flight (entries past the row's last block are read but never used).
   const bool spec_table = (!WL && a.windows == nullptr && a.window == 0);
+  bool spec0 = false;  // copy warp: the partition's first stage is already in flight
   if (warp == 0 && spec_table) {
     const int sj0 = (part * a.part_tokens) >> a.block_shift;
     const int sn = min(a.part_tokens / a.block_size + 2, a.max_blocks_per_seq - sj0);
     for (int i = lane; i < sn; i += 32)
       bt_s[i] = a.block_tables[(size_t)b * a.max_blocks_per_seq + sj0 + i];
+    // The first stage of a window-free partition starts at part * part_tokens
+    // whatever the lengths say, so its boxes go out now, before the lengths
+    // arrive.  Tokens past the row's end are masked like any stage's; table
+    // entries outside the pool are clamped into it, so every copy stays inside
+    // the tensor map (such an entry is still flagged below).
+    const int c0 = part * a.part_tokens;
+    if (a.spec_first_stage && c0 + TS <= a.max_blocks_per_seq * a.block_size) {
+      __syncwarp();
+      const int br = min(a.block_size, TS);
+      const int nitem0 = (TS / br) * 2;
+      const uint32_t bb = (uint32_t)br * T::ROW_BYTES;
+      uint32_t dst = 0;
+      int y = 0, isv = 0;
+      if (lane < nitem0) {
+        const int jb = lane >> 1;
+        isv = lane & 1;
+        const int bt0 = c0 + jb * br;
+        const int jj = bt0 >> a.block_shift;
+        const int phys = min(max(bt_s[jj - sj0], 0), a.num_blocks - 1);
+        y = (phys * a.num_kv_heads + kvh) * a.block_size + (bt0 - (jj << a.block_shift));
+        dst = isv * T::KV_BYTES + jb * bb;
+      }
+      if (lane == 0) mbar_arrive_expect_tx(smem_u32(&bars[0]), (uint32_t)nitem0 * bb);
+      __syncwarp();
+      if (lane < nitem0)
+        tma_load_3d_hint(smem_u32(smem) + dst,
+                         isv ? static_cast<const void*>(&tmv) : static_cast<const void*>(&tmk), 0,
+                         y, 0, smem_u32(&bars[0]), l2_evict_first_policy());
+      spec0 = true;
+    }
   }
-  if (L <= 0) return;
+  // A CTA that leaves with a speculative stage in flight first waits for it.
+  auto leave = [&]() {
+    if (spec0 && lane == 0) mbar_wait(smem_u32(&bars[0]), 0);
+  };
+  if (L <= 0) {
+    leave();
+    return;
+  }
   const bool lead = (part == 0 && slab == 0 && kvh == 0 && threadIdx.x == 0);
   if (L > S || w < 0 || S > a.max_blocks_per_seq * a.block_size) {
     if (lead) atomicOr(&g_pa_status, PA_DEV_BAD_ROW);
+    leave();
     return;
   }
   const int R = a.group * L;
@@ -709,10 +748,14 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
   const int nparts = (S - A + a.part_tokens - 1) / a.part_tokens;
   if (R > a.max_rows || nparts > a.max_parts) {
     if (lead) atomicOr(&g_pa_status, PA_DEV_HINT);
+    leave();
     return;
   }
   const int row0 = slab * a.slab_rows;
-  if (row0 >= R || part >= nparts) return;
+  if (row0 >= R || part >= nparts) {
+    leave();
+    return;
+  }
   const int Rs = min(a.slab_rows, R - row0);
   // Static schedule: this CTA's partition [p0, p1).  Work list: any stage of
   // the unit's span [A, S), so tokens are masked only at the span's ends.
@@ -894,7 +937,7 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
       raw = table_entry(st_n1);
     };
 
-    int k = 0;
+    int k = spec0 ? 1 : 0;
     bool ok = true;
     if constexpr (!WL) {
       for (; k < nst; ++k)

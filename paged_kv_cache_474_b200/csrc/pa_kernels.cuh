@@ -37,6 +37,10 @@ struct DecodeArgs {
   int max_rows;     // rows per unit the workspace holds
   int slab_rows;    // rows one CTA handles
   int num_slabs;    // CTAs per unit along grid.y (grid.y = H_kv * num_slabs)
+  // One-wave grids of window-free rows: each CTA issues its partition's first
+  // stage before the lengths arrive (the longest rows fill the grid, so few
+  // of those copies are for partitions past a row's end).
+  int spec_first_stage;
   // Work-list schedule (tensor-core kernel, one-wave cooperative grid): a
   // unit's CTAs claim its 64-token stages from a counter and merge their own
   // partials instead of a reduce kernel.
