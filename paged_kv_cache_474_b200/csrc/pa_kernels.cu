@@ -682,6 +682,11 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
     }
     fence_mbar_init();
   }
+  // Every thread sees the initialised barriers before any of them can use
+  // one.  With the early first stage (spec_first_stage) no warp waits for
+  // another after this point before the main loops, so the copy warp's wait
+  // for its table entries never holds up the compute warps' prologue.
+  __syncthreads();
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
   const int S = a.seq_lens[b];
@@ -765,7 +770,9 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
   const int jb0 = p0 >> a.block_shift;
   const int nbt = ((p1 - 1) >> a.block_shift) - jb0 + 1;
 
-  __syncthreads();
+  // Without the early first stage the warps meet once more here (measured a
+  // little faster on the multi-wave and windowed workloads).
+  if (!a.spec_first_stage) __syncthreads();
   // Let the reduce grid launch now; it waits for this grid's completion
   // before reading any partial.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
