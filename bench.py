@@ -174,7 +174,7 @@ def run_ours(args, rank, world, local_rank):
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
     stream = torch.cuda.current_stream()
-    wl = config_workload(args.config, device=device)
+    wl = config_workload(args.config, device=device, kv_dtype=args.kv_dtype)
     kv_bytes, qo_bytes = algorithmic_bytes(wl)
     call_bytes = kv_bytes + qo_bytes
 
@@ -251,7 +251,8 @@ def run_ours(args, rank, world, local_rank):
     kern_avg_ms = sum(kern_ms) / len(kern_ms)
     peak, peak_kind = measured_hbm_peak()
     achieved = call_bytes / (kern_avg_ms * 1e-3) / 1e9
-    traffic = traffic_from_profiles(kernel_source_hash(), CONFIG_TITLES[args.config])
+    title = CONFIG_TITLES[args.config] + ("" if args.kv_dtype == "bf16" else ", FP8 e4m3 KV")
+    traffic = traffic_from_profiles(kernel_source_hash(), title)
 
     # end to end through the host-buffer entry point
     e2e = run_e2e(args, wl, pa, torch, device, world)
@@ -269,9 +270,9 @@ def run_ours(args, rank, world, local_rank):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "bf16" if args.kv_dtype == "bf16" else "fp8_e4m3 KV, bf16 q/dst",
         "data": "synthetic",
-        "config": {"workload": CONFIG_TITLES[args.config],
+        "config": {"workload": title,
                    "kv_bytes_per_call": kv_bytes, "q_dst_bytes_per_call": qo_bytes,
                    "l2": "inputs larger than L2 (no flush between steps)",
                    "parallelism": f"replicas x{world} (rows shard, no collective)",
@@ -307,10 +308,10 @@ def run_e2e(args, wl, pa, torch, device, world):
     Lp = torch.from_numpy(L).pin_memory()
     Wp = None if W is None else torch.from_numpy(W).pin_memory()
     q_host = wl.q.cpu().contiguous().pin_memory()
-    out_host = torch.empty_like(q_host).pin_memory()
-    p = pa.make_params(batch=wl.batch, num_q_heads=wl.num_q_heads,
-                       num_kv_heads=wl.num_kv_heads, head_dim=wl.head_dim,
-                       num_blocks=wl.num_blocks, max_blocks_per_seq=wl.max_blocks_per_seq)
+    out_host = torch.empty(wl.q.shape, dtype=torch.bfloat16).pin_memory()
+    # the device call's parameters (operand types and scales), hints left to
+    # pa_decode_host, which computes them from the host lengths
+    p = pa.params_for(wl, hints=False)
     p.windows = None if Wp is None else Wp.data_ptr()
     n = pa.pa_host_workspace_size(p, wl.block_size, wl.window, Sp.data_ptr(), Lp.data_ptr())
     ws = torch.empty(n, dtype=torch.uint8, device=device)
@@ -339,7 +340,8 @@ def run_e2e(args, wl, pa, torch, device, world):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         el = float(t.item())
     kv, qo = algorithmic_bytes(wl)
-    h2d = q_host.numel() * 2 + bt.numel() * 4 + S.nbytes + L.nbytes + (0 if W is None else W.nbytes)
+    h2d = (q_host.numel() * q_host.element_size() + bt.numel() * 4 + S.nbytes + L.nbytes +
+           (0 if W is None else W.nbytes))
     d2h = out_host.numel() * 2
     return {"value": round((kv + qo) * args.steps * world / el / 1e9, 2), "unit": "GB/s",
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
@@ -554,6 +556,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--kv-dtype", choices=["bf16", "fp8_e4m3"], default="bf16",
+                    help="KV cache element type of the timed workload (FP8: per-tensor scaled e4m3)")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the per-config table and the CPU baseline")
     args = ap.parse_args()
