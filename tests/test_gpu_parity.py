@@ -324,16 +324,19 @@ def test_device_detects_rows_beyond_hints_and_bad_blocks():
     out = torch.zeros_like(wl.q)
     assert _raw_decode(wl, p, out) == pa.PA_OK
     assert pa.pa_device_status(clear=True) & pa.PA_DEV_HINT
-    # a block-table entry outside the pool is flagged, not dereferenced
-    bad = wl.block_tables.clone()
-    bad[1, 0] = wl.num_blocks + 5
-    wl2 = type(wl)(**{**wl.__dict__, "block_tables": bad})
-    p = pa.params_for(wl2)
-    ws = pa.alloc_workspace(p, 16)
-    if ws is not None:
-        p.workspace, p.workspace_bytes = ws.data_ptr(), ws.numel()
-    assert _raw_decode(wl2, p, out) == pa.PA_OK
-    assert pa.pa_device_status(clear=True) & pa.PA_DEV_BAD_BLOCK
+    # block-table entries outside the pool (above it, or negative) are flagged,
+    # not dereferenced, also in a partition's first stage, which this one-wave,
+    # window-free plan issues before the lengths arrive
+    for first, value in ((1, wl.num_blocks + 5), (0, -7)):
+        bad = wl.block_tables.clone()
+        bad[first, 0] = value
+        wl2 = type(wl)(**{**wl.__dict__, "block_tables": bad})
+        p = pa.params_for(wl2)
+        ws = pa.alloc_workspace(p, 16)
+        if ws is not None:
+            p.workspace, p.workspace_bytes = ws.data_ptr(), ws.numel()
+        assert _raw_decode(wl2, p, out) == pa.PA_OK
+        assert pa.pa_device_status(clear=True) & pa.PA_DEV_BAD_BLOCK
     # a row whose queryLen exceeds its seqLen is flagged when hints skip the host check
     lens = torch.tensor([900, 2], dtype=torch.int32, device="cuda:0")
     ql = torch.tensor([1, 3], dtype=torch.int32, device="cuda:0")
