@@ -745,7 +745,10 @@ int pa_decode_host(void* dst_host, const void* q_host, const void* kCache, const
     }
   }
   if (e == cudaSuccess && sa.n) e = pa::launch_stage(sa, st);
-  if (e != cudaSuccess) return fail(PA_ERR_CUDA, "host-to-device copy: %s", cudaGetErrorString(e));
+  if (e != cudaSuccess) {
+    cudaStreamSynchronize(st);  // copies already queued finish before the buffers go back
+    return fail(PA_ERR_CUDA, "host-to-device copy: %s", cudaGetErrorString(e));
+  }
   // Output: a mapped, 16-byte aligned dst is written by the kernels in place.
   void* dst_mapped = aligned16(dst_host) ? mapped_host(dst_host, dbytes_raw) : nullptr;
   if (dst_mapped) d_dst = static_cast<char*>(dst_mapped);
@@ -760,7 +763,14 @@ int pa_decode_host(void* dst_host, const void* q_host, const void* kCache, const
     rc = decode_impl(d_dst, d_q, kCache, vCache, reinterpret_cast<const int32_t*>(d_bt),
                      reinterpret_cast<const int32_t*>(d_S), reinterpret_cast<const int32_t*>(d_L),
                      scale, window, kvBlockSize, &dp, st, span, qlen);
-    if (rc) return rc;
+    if (rc) {
+      // the staging copies (and any kernel already launched) may still read
+      // or write the caller's host buffers: let them finish before returning
+      const std::string msg = g_err;
+      cudaStreamSynchronize(st);
+      g_err = msg;
+      return rc;
+    }
   }
   if (dbytes_raw && !dst_mapped)
     e = cudaMemcpyAsync(dst_host, d_dst, dbytes_raw, cudaMemcpyDeviceToHost, st);
