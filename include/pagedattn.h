@@ -182,6 +182,11 @@ typedef struct pa_plan_info {
  * PA_ERR_UNSUPPORTED for head_dim not in {64,128,256} or a block size outside
  * the set above; PA_ERR_WORKSPACE when split-K partials are needed and the
  * workspace is too small; PA_ERR_CUDA when a launch fails.
+ *
+ * With both hints set the call only enqueues kernels, so it can be recorded
+ * by a CUDA stream capture and replayed from a graph (replays read the
+ * buffers' current contents).  The first call on a device sets kernel
+ * attributes and queries occupancy; make it before capturing.
  */
 int pa_decode(void *dst, const void *q, const void *kCache, const void *vCache,
               const int32_t *blockTables, const int32_t *seqLens,

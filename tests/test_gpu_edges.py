@@ -2,7 +2,8 @@
 context (L == S), one-token rows, windows at and around the query length,
 rows without queries between rows with queries, and a large batch of short
 rows (thousands of (row, kv head) units and a long query-offset scan), on
-both kernel variants and with FP8 caches."""
+both kernel variants and with FP8 caches; and a call captured in a CUDA graph
+and replayed on new queries."""
 import numpy as np
 import pytest
 import torch
@@ -70,3 +71,43 @@ def test_large_batch_of_short_rows():
     rows = [b for b in range(3000) if L[b] > 0]
     sel = sample_queries(wl, 48, seed=62, rows=rows[-200:]) + sample_queries(wl, 16, seed=63)
     check_sampled(wl, out, sel, "3000 short rows")
+
+
+def test_decode_replays_inside_a_cuda_graph():
+    # With host hints set, pa_decode makes no synchronising call, so a stream
+    # capture records its launches (the partition kernel and the reduce, with
+    # their programmatic dependency); replays read the tensors' current values.
+    import paged_kv_cache_474_b200 as pa
+    from paged_kv_cache_474_b200.workloads import make_workload
+    wl = make_workload(seq_lens=[3000, 700, 45], query_lens=[1, 2, 1], num_q_heads=8,
+                       num_kv_heads=2, head_dim=128, block_size=16, seed=91, device="cuda:0")
+    p = pa.params_for(wl)
+    ws = pa.alloc_workspace(p, wl.block_size, device="cuda:0")
+    if ws is not None:
+        p.workspace, p.workspace_bytes = ws.data_ptr(), ws.numel()
+    out = torch.empty(wl.q.shape, dtype=torch.bfloat16, device="cuda:0")
+    q = wl.q.clone()
+
+    def call():
+        rc = pa.pa_decode(out.data_ptr(), q.data_ptr(), wl.k_cache.data_ptr(),
+                          wl.v_cache.data_ptr(), wl.block_tables.data_ptr(),
+                          wl.seq_lens.data_ptr(), wl.query_lens.data_ptr(), wl.scale,
+                          wl.window, wl.block_size, p, pa._stream_handle())
+        assert rc == pa.PA_OK, pa.pa_last_error()
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        call()   # first call on this device sets kernel attributes outside the capture
+    torch.cuda.current_stream().wait_stream(s)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call()
+    for seed in (1, 2, 3):
+        g = torch.Generator(device="cuda:0").manual_seed(seed)
+        q.copy_(torch.randn(q.shape, generator=g, device="cuda:0").to(torch.bfloat16))
+        graph.replay()
+        torch.cuda.synchronize()
+        ref = pa.decode(type(wl)(**{**wl.__dict__, "q": q}))
+        assert torch.equal(out, ref)
+    assert pa.pa_device_status(clear=True) == 0
