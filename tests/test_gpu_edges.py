@@ -3,7 +3,8 @@ context (L == S), one-token rows, windows at and around the query length,
 rows without queries between rows with queries, and a large batch of short
 rows (thousands of (row, kv head) units and a long query-offset scan), on
 both kernel variants and with FP8 caches; and a call captured in a CUDA graph
-and replayed on new queries."""
+and replayed on new queries; a decode loop whose inputs are written by the
+kernel just before each call."""
 import numpy as np
 import pytest
 import torch
@@ -110,4 +111,93 @@ def test_decode_replays_inside_a_cuda_graph():
         torch.cuda.synchronize()
         ref = pa.decode(type(wl)(**{**wl.__dict__, "q": q}))
         assert torch.equal(out, ref)
+    assert pa.pa_device_status(clear=True) == 0
+
+
+@pytest.mark.parametrize("variant", [pa.PA_VARIANT_AUTO, pa.PA_VARIANT_FMA])
+@pytest.mark.parametrize("window", [0, 200])
+def test_decode_loop_sees_inputs_written_just_before_each_call(variant, window):
+    # A decode loop with no host synchronisation.  Steps cycle through four
+    # orders, so that the kernel right before a call (the one a call may
+    # overlap while it drains) writes, in turn: seq_lens (after the new K/V
+    # token and q); the new K/V token (q is the previous call's dst); q; and
+    # nothing of this step (no new token, q is the previous dst, the previous
+    # call is the kernel before).  Each call's output is checked against the
+    # oracle at that step's lengths (positions written later lie past the
+    # step's context, so the final caches serve every step), and equals the
+    # same call made alone after a synchronise.
+    B, steps = 4, 8
+    appends = [t % 4 != 3 for t in range(steps)]
+    final = [900, 2500, 3100, 1700]
+    wl = make_workload(seq_lens=final, query_lens=[1] * B, num_q_heads=8, num_kv_heads=2,
+                       head_dim=128, block_size=16, window=window, seed=92, device="cuda:0")
+    p = pa.params_for(wl, force_variant=variant)  # hints from the final lengths bound every step
+    ws = pa.alloc_workspace(p, wl.block_size, device="cuda:0")
+    if ws is not None:
+        p.workspace, p.workspace_bytes = ws.data_ptr(), ws.numel()
+    g = torch.Generator(device="cuda:0").manual_seed(93)
+    new_k = torch.randn((steps, B, 2, 128), generator=g, device="cuda:0").to(torch.bfloat16)
+    new_v = torch.randn((steps, B, 2, 128), generator=g, device="cuda:0").to(torch.bfloat16)
+    q_src = torch.randn((steps,) + tuple(wl.q.shape), generator=g,
+                        device="cuda:0").to(torch.bfloat16)
+    # host-side positions of each step's new token, made before the loop so
+    # the loop launches only the kernels named above
+    start = [s - sum(appends) for s in final]
+    phys, off = [], []
+    n = 0
+    for t in range(steps):
+        n += appends[t]
+        tok = torch.tensor([s0 + n - 1 for s0 in start], dtype=torch.long)
+        phys.append(wl.block_tables.cpu()[torch.arange(B), tok // 16].long().to("cuda:0"))
+        off.append((tok % 16).to("cuda:0"))
+    sl = torch.tensor(start, dtype=torch.int32, device="cuda:0")
+    q_buf = torch.empty_like(wl.q)
+    torch.cuda.synchronize()
+    outs, qs, lens = [], [], []
+
+    def call(q, out, lengths):
+        rc = pa.pa_decode(out.data_ptr(), q.data_ptr(), wl.k_cache.data_ptr(),
+                          wl.v_cache.data_ptr(), wl.block_tables.data_ptr(),
+                          lengths.data_ptr(), wl.query_lens.data_ptr(), wl.scale,
+                          wl.window, wl.block_size, p, pa._stream_handle())
+        assert rc == pa.PA_OK, pa.pa_last_error()
+
+    def append(t):
+        wl.k_cache[phys[t], :, off[t], :] = new_k[t]
+        wl.v_cache[phys[t], :, off[t], :] = new_v[t]
+
+    def fresh_q(t):
+        torch.add(q_src[t], 0, out=q_buf)
+        return q_buf
+
+    for t in range(steps):
+        phase = t % 4
+        if phase == 0:
+            append(t)
+            q = fresh_q(t)
+            sl.add_(1)
+        elif phase == 1:
+            sl.add_(1)
+            q = outs[-1]
+            append(t)
+        elif phase == 2:
+            sl.add_(1)
+            append(t)
+            q = fresh_q(t)
+        else:
+            q = outs[-1]
+        out = torch.empty_like(wl.q)
+        call(q, out, sl)
+        outs.append(out)
+        qs.append(q.clone())  # stream-ordered after the call
+        lens.append(sl.clone())
+    torch.cuda.synchronize()
+    for t in range(steps):
+        wt = type(wl)(**{**wl.__dict__, "q": qs[t], "seq_lens": lens[t]})
+        check_full(wt, outs[t], f"decode loop step {t} window={window} variant={variant}")
+        alone = torch.empty_like(wl.q)
+        call(qs[t], alone, lens[t])
+        torch.cuda.synchronize()
+        assert torch.equal(alone, outs[t]), f"step {t}"
+    assert lens[-1].cpu().tolist() == final
     assert pa.pa_device_status(clear=True) == 0
