@@ -1,0 +1,88 @@
+"""GPU parity on seeded random configurations: head_dim, block size, GQA
+group, batch, lengths from one token to a few thousand, query lengths 0-5,
+no window / one window / per-row windows, bf16 or FP8 caches and queries,
+each kernel variant that supports the draw, forced partition counts and the
+no-hints path, every output element against the oracle.  The draws mix the
+shapes the named workloads use with combinations none of them has."""
+import numpy as np
+import pytest
+
+from tests.parity_helpers import check_full
+
+pa = pytest.importorskip("paged_kv_cache_474_b200")
+from paged_kv_cache_474_b200.workloads import make_workload  # noqa: E402
+
+NSEEDS = 160
+
+
+def draw(seed):
+    """One seeded configuration: (make_workload keywords, decode keywords)."""
+    g = np.random.default_rng(1000 + seed)
+    D = int(g.choice([64, 128, 128, 256]))
+    BS = int(g.choice([16, 16, 32, 64, 128, 256, 512, 1024]))
+    hkv = int(g.choice([1, 2, 4]))
+    group = int(g.choice([1, 2, 3, 4, 5, 8, 16, 32]))
+    B = int(g.integers(1, 7))
+    kind = g.choice(["tiny", "mid", "long", "longer"], size=B, p=[0.3, 0.35, 0.25, 0.1])
+    lo_hi = {"tiny": (1, 41), "mid": (41, 601), "long": (601, 3001), "longer": (3001, 12001)}
+    S = [int(g.integers(*lo_hi[k])) for k in kind]
+    L = [int(min(s, g.choice([0, 1, 1, 1, 2, 3, 5]))) for s in S]
+    if sum(L) == 0:
+        L[0] = 1
+    wmode = g.choice(["none", "one", "rows"])
+    window, windows = 0, None
+    if wmode == "one":
+        window = int(g.choice([1, 2, 7, 64, 500, 5000]))
+    elif wmode == "rows":
+        windows = [int(g.choice([0, 1, 3, 16, 100, 1000])) for _ in range(B)]
+    kv_fp8 = g.random() < 0.3
+    q_fp8 = g.random() < 0.15
+    fp8 = kv_fp8 or q_fp8
+    variants = [pa.PA_VARIANT_AUTO]
+    if not fp8 and D != 256:
+        variants.append(pa.PA_VARIANT_FMA)
+    if kv_fp8 and D == 128:
+        variants.append(pa.PA_VARIANT_TC)
+    variant = int(g.choice(variants))
+    parts = int(g.choice([0, 0, 0, 1, 2, 3, 7]))
+    hints = bool(g.random() < 0.8)
+    wl_kw = dict(seq_lens=S, query_lens=L, num_q_heads=hkv * group, num_kv_heads=hkv,
+                 head_dim=D, block_size=BS, window=window, windows=windows,
+                 dist=str(g.choice(["normal", "uniform"])), seed=2000 + seed,
+                 spare_blocks=int(g.integers(1, 4)), extra_table_cols=int(g.integers(0, 3)),
+                 kv_dtype="fp8_e4m3" if kv_fp8 else "bf16",
+                 q_dtype="fp8_e4m3" if q_fp8 else "bf16")
+    return wl_kw, dict(force_variant=variant, force_partitions=parts, hints=hints)
+
+
+def test_draws_cover_the_space_and_plan_on_the_host():
+    # the seeds below reach every head_dim, variant, dtype mix and window
+    # mode, and every draw is a valid call (the host plan accepts it)
+    draws = [draw(s) for s in range(NSEEDS)]
+    for w, d in draws:
+        wl = make_workload(**w)
+        p = pa.params_for(wl, hints=True, force_variant=d["force_variant"],
+                          force_partitions=d["force_partitions"])
+        rc, _ = pa.pa_plan(p, wl.block_size, num_sms=148, ctas_per_sm=2)
+        assert rc == pa.PA_OK, (w, d, pa.pa_last_error())
+    assert {w["head_dim"] for w, _ in draws} == {64, 128, 256}
+    assert {d["force_variant"] for _, d in draws} == {pa.PA_VARIANT_AUTO, pa.PA_VARIANT_FMA,
+                                                       pa.PA_VARIANT_TC}
+    assert {w["kv_dtype"] for w, _ in draws} == {"bf16", "fp8_e4m3"}
+    assert {w["q_dtype"] for w, _ in draws} == {"bf16", "fp8_e4m3"}
+    assert any(w["windows"] is not None for w, _ in draws)
+    assert any(w["window"] > 0 for w, _ in draws)
+    assert any(not d["hints"] for _, d in draws)
+    assert {w["block_size"] for w, _ in draws} >= {16, 1024}
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("seed", range(NSEEDS))
+def test_random_configuration(seed, cuda_device):
+    wl_kw, dec_kw = draw(seed)
+    wl = make_workload(**wl_kw)
+    pa.pa_device_status(clear=True)
+    out = pa.decode(wl.to("cuda:0"), **dec_kw)
+    assert pa.pa_device_status(clear=True) == 0
+    check_full(wl, out, f"seed {seed}: {wl_kw['head_dim']=} {wl_kw['block_size']=} "
+                        f"{wl_kw['seq_lens']=} {wl_kw['query_lens']=} {dec_kw}")
