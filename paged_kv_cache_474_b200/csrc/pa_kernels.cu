@@ -920,8 +920,19 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
     auto advance = [&](int kk, unsigned long long& pend, int& raw) {
       if (kk == 0 && lane == 0) {  // open this CTA's claims
         epoch_reset_if_stale(ctr, seen_ctr, a.epoch);
-        pendA = atomicAdd(ctr, 1ull);
-        pendB = atomicAdd(ctr, 1ull);
+        // Claims must resolve in the order their tickets were taken, so that
+        // a CTA's first out-of-range ticket comes after all its valid ones
+        // (the copies stop there).  The first claim resolves at stage
+        // kFixed - 3, on that stage's parity: the lower ticket goes there.
+        const unsigned long long t0 = atomicAdd(ctr, 1ull);
+        const unsigned long long t1 = atomicAdd(ctr, 1ull);
+        if constexpr (((kFixed - 3) & 1) == 0) {
+          pendA = t0;
+          pendB = t1;
+        } else {
+          pendB = t0;
+          pendA = t1;
+        }
         epoch_reset_if_stale(done, seen_done, a.epoch);
         s_dtouch = 1;
       }

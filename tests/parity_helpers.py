@@ -134,3 +134,15 @@ def scaled_workload(cfg, seed=1, **kw):
                              windows=[700 if b % 2 == 0 else 0 for b in range(6)],
                              seed=seed, **kw)
     raise ValueError(cfg)
+
+
+def host_buffer(arr, kind, offset=0):
+    """A host copy of ``arr`` (a CPU tensor): pinned (read in place by the
+    library's staging kernel) or pageable (copied), optionally starting
+    ``offset`` bytes into a larger buffer of the same kind."""
+    raw = arr.contiguous().view(torch.uint8).reshape(-1)
+    buf = torch.zeros(raw.numel() + offset + 16, dtype=torch.uint8)
+    if kind == "pinned":
+        buf = buf.pin_memory()
+    buf[offset:offset + raw.numel()] = raw
+    return buf, buf.data_ptr() + offset

@@ -10,7 +10,7 @@ import pytest
 import torch
 
 import oracle
-from tests.parity_helpers import (assert_close, check_full, check_sampled,
+from tests.parity_helpers import (assert_close, check_full, check_sampled, host_buffer,
                                   problem, sample_queries, scaled_workload, token_offsets)
 
 pytestmark = pytest.mark.gpu
@@ -206,18 +206,6 @@ def test_visible_ranges_match_oracle_exactly():
         assert np.array_equal(hi.cpu().numpy(), rhi)
 
 
-def _host_buffer(arr, kind, offset=0):
-    """A host copy of ``arr`` (a CPU tensor): pinned (read in place by the
-    library's staging kernel) or pageable (copied), optionally starting
-    ``offset`` bytes into a larger buffer of the same kind."""
-    raw = arr.contiguous().view(torch.uint8).reshape(-1)
-    buf = torch.zeros(raw.numel() + offset + 16, dtype=torch.uint8)
-    if kind == "pinned":
-        buf = buf.pin_memory()
-    buf[offset:offset + raw.numel()] = raw
-    return buf, buf.data_ptr() + offset
-
-
 # kinds of q / tables+lengths+windows / dst host buffers, and byte offsets of
 # q, tables and dst inside their buffers (offsets that break 16-byte or 4-byte
 # alignment take the narrower staging copies or the copy-back path)
@@ -243,7 +231,7 @@ def test_host_entry_point_matches_device_path(cfg, case):
     keep = []
 
     def host(t, kind, off=0):
-        buf, ptr = _host_buffer(t, kind, off)
+        buf, ptr = host_buffer(t, kind, off)
         keep.append(buf)
         return ptr
     S = host(wl.seq_lens, kt)
@@ -255,7 +243,7 @@ def test_host_entry_point_matches_device_path(cfg, case):
     p.workspace, p.workspace_bytes = ws.data_ptr(), n
     q = host(wl.q, kq, oq)
     bt = host(wl.block_tables, kt, ot)
-    out_buf, out_ptr = _host_buffer(torch.full(wl.q.shape, float("nan"), dtype=torch.bfloat16),
+    out_buf, out_ptr = host_buffer(torch.full(wl.q.shape, float("nan"), dtype=torch.bfloat16),
                                     kd, od)
     for _ in range(2):   # twice: the second call overwrites the first's output in place
         rc = pa.pa_decode_host(out_ptr, q, d.k_cache.data_ptr(), d.v_cache.data_ptr(), bt, S, L,
@@ -447,6 +435,31 @@ def test_work_list_workspace_needs_no_initialisation(fill):
     for _ in range(3 if fill == "reuse" else 1):
         out = pa.decode(d, workspace=ws, schedule=pa.PA_SCHED_WORKLIST)
         assert_close(out.float().cpu().numpy(), ref, f"work list workspace {fill}")
+
+
+@pytest.mark.parametrize("parts", [1, 2, 3])
+@pytest.mark.parametrize("head_dim,kv_dtype", [(64, "bf16"), (64, "fp8_e4m3"), (128, "bf16"),
+                                               (128, "fp8_e4m3")])
+def test_work_list_stage_counts_around_the_fixed_runs(head_dim, kv_dtype, parts):
+    # Each CTA owns (ring depth + 2) stages outright and claims the rest from
+    # the unit's counter.  Rows of parts x that many stages, give or take
+    # three (ragged last stage), put the first claims and the first claim past
+    # the end on either ring parity; the rings here are 3, 4 and 8 deep.
+    probe = make_workload(seq_lens=[64], query_lens=[1], num_q_heads=8, num_kv_heads=2,
+                          head_dim=head_dim, block_size=16, kv_dtype=kv_dtype)
+    rc, info = pa.pa_plan(pa.params_for(probe, force_partitions=1,
+                                        schedule=pa.PA_SCHED_WORKLIST), 16)
+    assert rc == pa.PA_OK, pa.pa_last_error()
+    fixed = parts * (info.stages + 2)
+    S = [n * 64 - 8 for n in range(fixed - 3, fixed + 4)]
+    wl = make_workload(seq_lens=S, query_lens=[1] * len(S), num_q_heads=8, num_kv_heads=2,
+                       head_dim=head_dim, block_size=16, seed=78, kv_dtype=kv_dtype)
+    d = dev(wl)
+    _, plan = pa.pa_plan(pa.params_for(d, force_partitions=parts,
+                                       schedule=pa.PA_SCHED_WORKLIST), 16)
+    assert plan.worklist and plan.stages == info.stages
+    out = pa.decode(d, force_partitions=parts, schedule=pa.PA_SCHED_WORKLIST)
+    check_full(wl, out, f"work list D={head_dim} {kv_dtype} parts={parts}")
 
 
 def test_work_list_schedule_refuses_multi_wave_grids():

@@ -6,8 +6,9 @@ no-hints path, every output element against the oracle.  The draws mix the
 shapes the named workloads use with combinations none of them has."""
 import numpy as np
 import pytest
+import torch
 
-from tests.parity_helpers import check_full
+from tests.parity_helpers import check_full, host_buffer
 
 pa = pytest.importorskip("paged_kv_cache_474_b200")
 from paged_kv_cache_474_b200.workloads import make_workload  # noqa: E402
@@ -74,6 +75,16 @@ def test_draws_cover_the_space_and_plan_on_the_host():
     assert any(w["window"] > 0 for w, _ in draws)
     assert any(not d["hints"] for _, d in draws)
     assert {w["block_size"] for w, _ in draws} >= {16, 1024}
+    # the work-list schedule (one-wave grids only) accepts a good share of them
+    ok = 0
+    for w, d in draws:
+        if d["force_variant"] != pa.PA_VARIANT_AUTO:
+            continue
+        wl = make_workload(**w)
+        p = pa.params_for(wl, force_partitions=d["force_partitions"],
+                          schedule=pa.PA_SCHED_WORKLIST)
+        ok += pa.pa_plan(p, wl.block_size, num_sms=148, ctas_per_sm=2)[0] == pa.PA_OK
+    assert ok >= 40
 
 
 @pytest.mark.gpu
@@ -86,3 +97,66 @@ def test_random_configuration(seed, cuda_device):
     assert pa.pa_device_status(clear=True) == 0
     check_full(wl, out, f"seed {seed}: {wl_kw['head_dim']=} {wl_kw['block_size']=} "
                         f"{wl_kw['seq_lens']=} {wl_kw['query_lens']=} {dec_kw}")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("seed", range(0, NSEEDS, 4))
+def test_random_configuration_host_entry(seed, cuda_device):
+    # pa_decode_host with q, lengths, tables, windows and dst in host memory
+    # (pinned or pageable, drawn per buffer): the same bits as the device
+    # entry point with the same plan, and within tolerance of the oracle
+    wl_kw, dec_kw = draw(seed)
+    wl = make_workload(**wl_kw)
+    d = wl.to("cuda:0")
+    ref = pa.decode(d, force_variant=dec_kw["force_variant"],
+                    force_partitions=dec_kw["force_partitions"])
+    g = np.random.default_rng(3000 + seed)
+    kq, kt, kd = (str(g.choice(["pinned", "pageable"])) for _ in range(3))
+    keep = []
+
+    def host(t, kind):
+        buf, ptr = host_buffer(t, kind)
+        keep.append(buf)
+        return ptr
+    p = pa.params_for(wl, hints=False, force_variant=dec_kw["force_variant"],
+                      force_partitions=dec_kw["force_partitions"])
+    S = host(wl.seq_lens, kt)
+    L = host(wl.query_lens, kt)
+    if wl.windows is not None:
+        p.windows = host(wl.windows, kt)
+    n = pa.pa_host_workspace_size(p, wl.block_size, wl.window, S, L)
+    ws = torch.empty(max(n, 1), dtype=torch.uint8, device="cuda:0")
+    p.workspace, p.workspace_bytes = ws.data_ptr(), n
+    out_buf, out_ptr = host_buffer(torch.full(wl.q.shape, float("nan"), dtype=torch.bfloat16), kd)
+    pa.pa_device_status(clear=True)
+    rc = pa.pa_decode_host(out_ptr, host(wl.q, kq), d.k_cache.data_ptr(), d.v_cache.data_ptr(),
+                           host(wl.block_tables, kt), S, L, wl.scale, wl.window, wl.block_size,
+                           p, pa._stream_handle())
+    assert rc == pa.PA_OK, pa.pa_last_error()
+    assert pa.pa_device_status(clear=True) == 0
+    got = out_buf[:ref.numel() * 2].view(torch.bfloat16).reshape(ref.shape)
+    assert torch.equal(got, ref.cpu()), f"seed {seed} ({kq}, {kt}, {kd})"
+    check_full(wl, got, f"host entry seed {seed}")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("seed", range(NSEEDS))
+def test_random_configuration_work_list(seed, cuda_device):
+    # the work-list schedule on every draw it accepts (the default variant,
+    # grids of one wave on this GPU)
+    wl_kw, dec_kw = draw(seed)
+    if dec_kw["force_variant"] != pa.PA_VARIANT_AUTO:
+        pytest.skip("the work-list schedule runs on the default variant only")
+    wl = make_workload(**wl_kw)
+    d = wl.to("cuda:0")
+    p = pa.params_for(d, force_partitions=dec_kw["force_partitions"],
+                      schedule=pa.PA_SCHED_WORKLIST)
+    rc, _ = pa.pa_plan(p, wl.block_size)
+    if rc == pa.PA_ERR_UNSUPPORTED:
+        pytest.skip("grid of more than one wave")
+    assert rc == pa.PA_OK, pa.pa_last_error()
+    pa.pa_device_status(clear=True)
+    out = pa.decode(d, force_partitions=dec_kw["force_partitions"],
+                    schedule=pa.PA_SCHED_WORKLIST)
+    assert pa.pa_device_status(clear=True) == 0
+    check_full(wl, out, f"work list seed {seed}")
