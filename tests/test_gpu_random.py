@@ -56,6 +56,48 @@ def draw(seed):
     return wl_kw, dict(force_variant=variant, force_partitions=parts, hints=hints)
 
 
+def draw_wide(seed):
+    """A wider seeded configuration: up to 48 rows, query lengths up to 16
+    (MTP and prefill chunks), windows at and around the query length, log-
+    uniform context lengths; the oracle's work is capped by shortening rows."""
+    g = np.random.default_rng(5000 + seed)
+    D = int(g.choice([64, 128, 256]))
+    BS = int(g.choice([16, 32, 64, 128, 256, 512, 1024]))
+    hkv = int(g.choice([1, 2, 8]))
+    group = int(g.choice([1, 2, 4, 6, 8, 12, 16]))
+    B = int(g.integers(1, 49))
+    S = [int(np.exp(g.uniform(0.0, np.log(6000.0)))) + 1 for _ in range(B)]
+    L = [int(min(s, 1 if g.random() < 0.5 else g.integers(0, 17))) for s in S]
+    if sum(L) == 0:
+        L[0] = 1
+    windows = None
+    if g.random() < 0.6:
+        windows = [int(g.choice([0, 1, max(1, l - 1), max(1, l), l + 1, 50, 2000]))
+                   for l in L]
+    budget = 4e8 / (hkv * group * D)
+    while sum(l * min(s, (w or s) + l) for s, l, w in
+              zip(S, L, windows or [0] * B)) > budget:
+        S = [max(l, s // 2) for s, l in zip(S, L)]
+    kv_fp8 = g.random() < 0.3
+    q_fp8 = g.random() < 0.1
+    fp8 = kv_fp8 or q_fp8
+    variants = [pa.PA_VARIANT_AUTO]
+    if not fp8 and D != 256:
+        variants.append(pa.PA_VARIANT_FMA)
+    if kv_fp8 and D == 128:
+        variants.append(pa.PA_VARIANT_TC)
+    wl_kw = dict(seq_lens=S, query_lens=L, num_q_heads=hkv * group, num_kv_heads=hkv,
+                 head_dim=D, block_size=BS, windows=windows, seed=6000 + seed,
+                 kv_dtype="fp8_e4m3" if kv_fp8 else "bf16",
+                 q_dtype="fp8_e4m3" if q_fp8 else "bf16")
+    return wl_kw, dict(force_variant=int(g.choice(variants)),
+                       force_partitions=int(g.choice([0, 0, 2, 5])),
+                       hints=bool(g.random() < 0.8))
+
+
+NWIDE = 64
+
+
 def test_draws_cover_the_space_and_plan_on_the_host():
     # the seeds below reach every head_dim, variant, dtype mix and window
     # mode, and every draw is a valid call (the host plan accepts it)
@@ -85,6 +127,15 @@ def test_draws_cover_the_space_and_plan_on_the_host():
                           schedule=pa.PA_SCHED_WORKLIST)
         ok += pa.pa_plan(p, wl.block_size, num_sms=148, ctas_per_sm=2)[0] == pa.PA_OK
     assert ok >= 40
+    wide = [draw_wide(s) for s in range(NWIDE)]
+    for w, d in wide:
+        wl = make_workload(**w)
+        p = pa.params_for(wl, force_variant=d["force_variant"],
+                          force_partitions=d["force_partitions"])
+        rc, _ = pa.pa_plan(p, wl.block_size, num_sms=148, ctas_per_sm=2)
+        assert rc == pa.PA_OK, (w, d, pa.pa_last_error())
+    assert max(max(w["query_lens"]) for w, _ in wide) >= 12
+    assert max(len(w["seq_lens"]) for w, _ in wide) >= 40
 
 
 @pytest.mark.gpu
@@ -160,3 +211,14 @@ def test_random_configuration_work_list(seed, cuda_device):
                     schedule=pa.PA_SCHED_WORKLIST)
     assert pa.pa_device_status(clear=True) == 0
     check_full(wl, out, f"work list seed {seed}")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("seed", range(NWIDE))
+def test_wide_random_configuration(seed, cuda_device):
+    wl_kw, dec_kw = draw_wide(seed)
+    wl = make_workload(**wl_kw)
+    pa.pa_device_status(clear=True)
+    out = pa.decode(wl.to("cuda:0"), **dec_kw)
+    assert pa.pa_device_status(clear=True) == 0
+    check_full(wl, out, f"wide seed {seed}: {dec_kw}")
