@@ -146,3 +146,36 @@ def host_buffer(arr, kind, offset=0):
         buf = buf.pin_memory()
     buf[offset:offset + raw.numel()] = raw
     return buf, buf.data_ptr() + offset
+
+
+def poison_outside_spans(wl: Workload):
+    """Writes NaN (bf16 NaN, or the e4m3 NaN code 0x7F) into every cache
+    position no query token may see: before each row's earliest visible
+    position, past its last token in its last block, and in every block no
+    row uses; and puts out-of-pool entries (alternately too large and
+    negative) in the block-table slots past each row's last block.  In
+    place, on the workload's own tensors (CPU)."""
+    nan = 0x7F if wl.kv_fp8 else float("nan")
+    S = wl.seq_lens.tolist()
+    L = wl.query_lens.tolist()
+    W = wl.windows.tolist() if wl.windows is not None else [wl.window] * len(S)
+    bs = wl.block_size
+    for b in range(len(S)):
+        nb = (S[b] + bs - 1) // bs
+        first = max(0, S[b] - L[b] + 1 - W[b]) if (W[b] > 0 and L[b] > 0) else 0
+        if L[b] <= 0:
+            first = S[b]  # no query: nothing of the row is visible
+        dead = list(range(0, first)) + list(range(S[b], nb * bs))
+        if dead:
+            t = torch.tensor(dead, dtype=torch.long)
+            blk = wl.block_tables[b, t // bs].long()
+            wl.k_cache[blk, :, t % bs] = nan
+            wl.v_cache[blk, :, t % bs] = nan
+        cols = wl.block_tables.shape[1]
+        for j in range(nb, cols):
+            wl.block_tables[b, j] = 10 ** 6 + j if j % 2 == 0 else -7 - j
+    used = set(int(x) for x in wl.block_tables.flatten().tolist() if 0 <= x < wl.num_blocks)
+    for blk in range(wl.num_blocks):
+        if blk not in used:
+            wl.k_cache[blk] = nan
+            wl.v_cache[blk] = nan

@@ -3,12 +3,18 @@ group, batch, lengths from one token to a few thousand, query lengths 0-5,
 no window / one window / per-row windows, bf16 or FP8 caches and queries,
 each kernel variant that supports the draw, forced partition counts and the
 no-hints path, every output element against the oracle.  The draws mix the
-shapes the named workloads use with combinations none of them has."""
+shapes the named workloads use with combinations none of them has.  Subsets
+of the draws also run through the host entry point, on the work-list
+schedule, and with every position no query may see poisoned (NaN, and
+out-of-pool table slots past each row); a second, wider family of draws
+takes up to 48 rows and query lengths up to 16."""
 import numpy as np
 import pytest
 import torch
 
-from tests.parity_helpers import check_full, host_buffer
+import oracle
+from tests.parity_helpers import (assert_close, check_full, host_buffer, poison_outside_spans,
+                                  problem)
 
 pa = pytest.importorskip("paged_kv_cache_474_b200")
 from paged_kv_cache_474_b200.workloads import make_workload  # noqa: E402
@@ -136,6 +142,12 @@ def test_draws_cover_the_space_and_plan_on_the_host():
         assert rc == pa.PA_OK, (w, d, pa.pa_last_error())
     assert max(max(w["query_lens"]) for w, _ in wide) >= 12
     assert max(len(w["seq_lens"]) for w, _ in wide) >= 40
+    # poisoning touches only positions no query sees: the oracle is unchanged
+    for w, _ in draws[::8]:
+        wl = make_workload(**w)
+        ref = oracle.decode(problem(wl))
+        poison_outside_spans(wl)
+        assert np.array_equal(oracle.decode(problem(wl)), ref)
 
 
 @pytest.mark.gpu
@@ -222,3 +234,19 @@ def test_wide_random_configuration(seed, cuda_device):
     out = pa.decode(wl.to("cuda:0"), **dec_kw)
     assert pa.pa_device_status(clear=True) == 0
     check_full(wl, out, f"wide seed {seed}: {dec_kw}")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("seed", range(0, NSEEDS, 2))
+def test_random_configuration_never_reads_outside_spans(seed, cuda_device):
+    # every position no query may see holds NaN and every table slot past a
+    # row's blocks points outside the pool: outputs match the oracle on the
+    # clean inputs, and no bad block is flagged (those slots are never used)
+    wl_kw, dec_kw = draw(seed)
+    wl = make_workload(**wl_kw)
+    ref = oracle.decode(problem(wl))
+    poison_outside_spans(wl)
+    pa.pa_device_status(clear=True)
+    out = pa.decode(wl.to("cuda:0"), **dec_kw)
+    assert pa.pa_device_status(clear=True) == 0
+    assert_close(out.float().cpu().numpy(), ref, f"poisoned seed {seed}: {dec_kw}")
