@@ -135,7 +135,9 @@ typedef struct pa_params {
      * fits the GPU at once (PA_ERR_UNSUPPORTED otherwise, PA_ERR_CUDA if the
      * cooperative launch is refused).  The counters are tagged with a
      * per-call epoch and need no initialisation; calls that share a
-     * workspace must not overlap.  Results can differ from the static
+     * workspace must not overlap, and a call on a stream that is being
+     * captured into a CUDA graph fails with PA_ERR_UNSUPPORTED (a replay
+     * would repeat the epoch).  Results can differ from the static
      * schedule's in the last bits (the stages' grouping depends on timing),
      * and it measures slower on the named workloads, so it is opt-in. */
     int schedule;
@@ -185,7 +187,7 @@ typedef struct pa_plan_info {
  *
  * With both hints set the call only enqueues kernels, so it can be recorded
  * by a CUDA stream capture and replayed from a graph (replays read the
- * buffers' current contents).  The first call on a device sets kernel
+ * buffers' current contents); the work-list schedule is the exception.  The first call on a device sets kernel
  * attributes and queries occupancy; make it before capturing.
  */
 int pa_decode(void *dst, const void *q, const void *kCache, const void *vCache,

@@ -494,6 +494,12 @@ int decode_impl(void* dst, const void* q, const void* kCache, const void* vCache
     a.ws_lse = reinterpret_cast<float*>(ws);
     a.ws_o = reinterpret_cast<float*>(ws + pl.lse_bytes);
     if (in.worklist) {
+      // A graph replay would repeat the epoch recorded at capture, and a
+      // replay's counters would then look current from the start.
+      cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+      if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone)
+        return fail(PA_ERR_UNSUPPORTED,
+                    "the work-list schedule cannot be captured in a CUDA graph (per-call epoch)");
       static std::atomic<unsigned int> epochs{0};
       unsigned int e = ++epochs;
       if (e == 0) e = ++epochs;  // 0 is never a live epoch

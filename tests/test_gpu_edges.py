@@ -201,3 +201,32 @@ def test_decode_loop_sees_inputs_written_just_before_each_call(variant, window):
         assert torch.equal(alone, outs[t]), f"step {t}"
     assert lens[-1].cpu().tolist() == final
     assert pa.pa_device_status(clear=True) == 0
+
+
+def test_work_list_schedule_refuses_stream_capture():
+    # its counters carry a per-call epoch that a graph replay would repeat
+    wl = make_workload(seq_lens=[3000, 700], query_lens=[1, 1], num_q_heads=8, num_kv_heads=2,
+                       head_dim=128, block_size=16, seed=94, device="cuda:0")
+    p = pa.params_for(wl, schedule=pa.PA_SCHED_WORKLIST)
+    ws = pa.alloc_workspace(p, wl.block_size, device="cuda:0")
+    p.workspace, p.workspace_bytes = ws.data_ptr(), ws.numel()
+    out = torch.empty(wl.q.shape, dtype=torch.bfloat16, device="cuda:0")
+
+    def call():
+        return pa.pa_decode(out.data_ptr(), wl.q.data_ptr(), wl.k_cache.data_ptr(),
+                            wl.v_cache.data_ptr(), wl.block_tables.data_ptr(),
+                            wl.seq_lens.data_ptr(), wl.query_lens.data_ptr(), wl.scale,
+                            wl.window, wl.block_size, p, pa._stream_handle())
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        assert call() == pa.PA_OK, pa.pa_last_error()  # eager: fine
+    torch.cuda.current_stream().wait_stream(s)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        out.zero_()
+        rc = call()
+    assert rc == pa.PA_ERR_UNSUPPORTED and "graph" in pa.pa_last_error()
+    graph.replay()
+    torch.cuda.synchronize()
+    assert pa.pa_device_status(clear=True) == 0

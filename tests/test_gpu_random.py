@@ -250,3 +250,46 @@ def test_random_configuration_never_reads_outside_spans(seed, cuda_device):
     out = pa.decode(wl.to("cuda:0"), **dec_kw)
     assert pa.pa_device_status(clear=True) == 0
     assert_close(out.float().cpu().numpy(), ref, f"poisoned seed {seed}: {dec_kw}")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("seed", range(0, NSEEDS, 5))
+def test_random_configuration_replays_in_a_cuda_graph(seed, cuda_device):
+    # with hints set a call only enqueues kernels: captured once, replayed on
+    # new queries, it gives the same bits as an eager call on those queries
+    wl_kw, dec_kw = draw(seed)
+    wl = make_workload(**wl_kw).to("cuda:0")
+    kw = dict(force_variant=dec_kw["force_variant"], force_partitions=dec_kw["force_partitions"])
+    p = pa.params_for(wl, **kw)
+    ws = pa.alloc_workspace(p, wl.block_size, device="cuda:0")
+    if ws is not None:
+        p.workspace, p.workspace_bytes = ws.data_ptr(), ws.numel()
+    q = wl.q.clone()
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda:0")
+
+    def call():
+        rc = pa.pa_decode(out.data_ptr(), q.data_ptr(), wl.k_cache.data_ptr(),
+                          wl.v_cache.data_ptr(), wl.block_tables.data_ptr(),
+                          wl.seq_lens.data_ptr(), wl.query_lens.data_ptr(), wl.scale,
+                          wl.window, wl.block_size, p, pa._stream_handle())
+        assert rc == pa.PA_OK, pa.pa_last_error()
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        call()  # the first call on a device sets kernel attributes outside the capture
+    torch.cuda.current_stream().wait_stream(s)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        call()
+    g = torch.Generator(device="cuda:0").manual_seed(seed)
+    for k in (1, 2):
+        if q.dtype == torch.uint8:  # FP8 codes: other valid codes, the heads rotated
+            q.copy_(wl.q.roll(k, 1))
+        else:
+            q.copy_(torch.randn(q.shape, generator=g, device="cuda:0").to(torch.bfloat16))
+        graph.replay()
+        torch.cuda.synchronize()
+        eager = pa.decode(type(wl)(**{**wl.__dict__, "q": q.clone()}), **kw)
+        assert torch.equal(out, eager), f"seed {seed} replay {k}"
+    assert pa.pa_device_status(clear=True) == 0
