@@ -2,7 +2,8 @@
 
 Each test fixes the oracle to a fact from the pages or from mathematics:
   - brute force: PyTorch's float64 CPU scaled_dot_product_attention with an
-    explicit boolean mask, and an independent pure-Python loop;
+    explicit boolean mask (on fixed cases and on 24 seeded random shapes,
+    windows and dtypes), and an independent pure-Python loop;
   - window = context (or more) equals unlimited, and window 0 is full causal
     (gllm PR #116 "feat(backend): sliding-window PagedAttention",
     "Verification": "Window = context matches unlimited");
@@ -474,3 +475,39 @@ def test_fp8_query_scale_acts_on_the_logits():
     a = oracle.decode(oracle.Problem(*args, w.scale * 1.3, q_scale=w.q_scale, **kw))
     b = oracle.decode(oracle.Problem(*args, w.scale, q_scale=w.q_scale * 1.3, **kw))
     assert np.max(np.abs(a - b)) <= 1e-13
+
+
+def random_pin_workload(seed):
+    """Seeded random shapes for the SDPA pin: head_dim 8-256, block sizes 1-1024,
+    GQA groups 1-8 over 1-3 kv heads, 1-5 rows of 1-600 tokens with 0-5
+    query tokens, no window / one window / per-row windows, bf16 or FP8."""
+    g = np.random.default_rng(700 + seed)
+    B = int(g.integers(1, 6))
+    S = [int(g.integers(1, 601)) for _ in range(B)]
+    L = [int(min(s, g.integers(0, 6))) for s in S]
+    if sum(L) == 0:
+        L[0] = 1
+    hkv = int(g.choice([1, 2, 3]))
+    mode = g.choice(["none", "one", "rows"])
+    window = int(g.choice([1, 3, 50])) if mode == "one" else 0
+    windows = [int(g.choice([0, 1, 2, 17, 400])) for _ in range(B)] if mode == "rows" else None
+    w = make_workload(seq_lens=S, query_lens=L, num_q_heads=hkv * int(g.choice([1, 2, 5, 8])),
+                      num_kv_heads=hkv, head_dim=int(g.choice([8, 64, 128, 256])),
+                      block_size=int(g.choice([1, 4, 16, 1024])), window=window,
+                      windows=windows, dist=str(g.choice(["normal", "uniform"])),
+                      seed=800 + seed, scale=float(g.uniform(0.05, 0.5)),
+                      kv_dtype="fp8_e4m3" if g.random() < 0.3 else "bf16",
+                      q_dtype="fp8_e4m3" if g.random() < 0.15 else "bf16")
+    return w, (lambda b: windows[b]) if windows is not None else (lambda b: window)
+
+
+@pytest.mark.parametrize("seed", range(24))
+def test_random_shapes_match_torch_sdpa(seed):
+    # the dense-gather SDPA pin over random shapes, windows and dtypes, and
+    # the split-K form at a random partition count
+    w, wof = random_pin_workload(seed)
+    pr = problem_of(w)
+    got = oracle.decode(pr)
+    assert np.max(np.abs(got - sdpa_reference(w, wof))) <= 1e-12
+    parts = int(np.random.default_rng(seed).integers(2, 9))
+    assert np.max(np.abs(oracle.decode(pr, parts=parts) - got)) <= 1e-12
