@@ -27,6 +27,8 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "pa_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
+# Tests that plant a slip in a copy of the oracle point this at their build.
+_LIB_OVERRIDE = os.environ.get("PA_ORACLE_LIB")
 _lock = threading.Lock()
 _lib = None
 
@@ -48,8 +50,7 @@ def _load():
     global _lib
     with _lock:
         if _lib is None:
-            build()
-            lib = ctypes.CDLL(_LIB)
+            lib = ctypes.CDLL(_LIB_OVERRIDE or build())
             P = ctypes.c_void_p
             I = ctypes.c_int
             D = ctypes.c_double
