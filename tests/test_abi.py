@@ -299,3 +299,32 @@ def test_plan_work_list_schedule():
     assert rc == pa.PA_ERR_UNSUPPORTED
     one_shot = plan(schedule=pa.PA_SCHED_WORKLIST, max_span_hint=50)
     assert one_shot.one_shot and not one_shot.worklist and one_shot.workspace_bytes == 0
+
+
+def test_header_is_plain_c_and_matches_the_binding(tmp_path):
+    # tests/c_abi_check.c uses the header from C11 (pedantic, warnings as
+    # errors), links the library and calls its host-only entry points; its
+    # results equal the same calls through the binding
+    import subprocess
+    libdir = os.path.dirname(pa.LIB_PATH)
+    exe = tmp_path / "c_abi_check"
+    subprocess.run(["gcc", "-std=c11", "-pedantic", "-Wall", "-Wextra", "-Werror",
+                    "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c_abi_check.c"), "-o", str(exe),
+                    "-L", libdir, "-lpagedattn", f"-Wl,-rpath,{libdir}"], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout
+    lines = dict(line.split(" ", 1) for line in out.strip().splitlines())
+    S, L, W = [300, 40, 7], [5, 1, 3], [16, 100, 2]
+    span, qlen = pa.pa_extents_host(S, L, windows=W)
+    assert lines["extents"] == f"{span} {qlen}"
+    win = np.array(W, dtype=np.int32)
+    p = pa.make_params(batch=3, num_q_heads=8, num_kv_heads=2, head_dim=128, num_blocks=64,
+                       max_blocks_per_seq=19, max_span_hint=span, max_query_len_hint=qlen)
+    p.windows = win.ctypes.data
+    rc, info = pa.pa_plan(p, 16, num_sms=148, ctas_per_sm=2)
+    assert rc == pa.PA_OK
+    assert lines["plan"] == " ".join(str(x) for x in (
+        info.variant, info.partition_tokens, info.max_partitions, info.one_shot,
+        info.max_rows, info.grid_x, info.grid_y, info.grid_z, info.workspace_bytes))
+    assert lines["refused"] == f"{pa.PA_ERR_UNSUPPORTED} 1"
+    assert lines["version"] == pa.pa_version()
