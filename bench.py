@@ -523,13 +523,16 @@ def run_reference(args, rank, world):
     wl = config_workload(args.config, device="cpu")
     # per step: every row whose oracle pass fits ~2 s, so K+W steps end in minutes
     rows = _rows_for_budget(wl, 2.0)
+    # Under torchrun every process starts with OMP_NUM_THREADS=1, but only this
+    # rank works: give the oracle all of the host's cores, as at N=1.
+    nthreads = len(os.sched_getaffinity(0)) if world > 1 else 0
     for _ in range(args.warmup):
-        oracle_sample_run(wl, rows)
+        oracle_sample_run(wl, rows, nthreads)
     tot_t = 0.0
     tot_b = 0
     thr = 1
     for _ in range(args.steps):
-        t, b, thr = oracle_sample_run(wl, rows)
+        t, b, thr = oracle_sample_run(wl, rows, nthreads)
         tot_t += t
         tot_b += b
     value = tot_b / tot_t / 1e9
