@@ -328,3 +328,57 @@ def test_header_is_plain_c_and_matches_the_binding(tmp_path):
         info.max_rows, info.grid_x, info.grid_y, info.grid_z, info.workspace_bytes))
     assert lines["refused"] == f"{pa.PA_ERR_UNSUPPORTED} 1"
     assert lines["version"] == pa.pa_version()
+
+
+def test_plan_invariants_on_random_params():
+    # 600 seeded draws of shapes, hints, variants, partition counts and KV
+    # dtypes: every plan the host accepts keeps the dispatcher's promises, and
+    # the only refusals are the documented ones
+    g = np.random.default_rng(5)
+    align = lambda x: (x + 255) // 256 * 256
+    accepted = 0
+    for _ in range(600):
+        D = int(g.choice([64, 128, 256]))
+        BS = int(g.choice([16, 32, 64, 128, 256, 512, 1024]))
+        hkv, grp = int(g.choice([1, 2, 4, 8])), int(g.choice([1, 2, 3, 4, 8, 16]))
+        B, mbps, qlen = int(g.integers(1, 3000)), int(g.integers(1, 4096)), int(g.integers(1, 17))
+        span = int(g.integers(1, mbps * BS + 1))
+        fp8 = bool(g.random() < 0.3)
+        fv, fp = int(g.choice([0, 0, 0, pa.PA_VARIANT_FMA])), int(g.choice([0, 0, 0, 2, 7, 100]))
+        p = pa.make_params(batch=B, num_q_heads=hkv * grp, num_kv_heads=hkv, head_dim=D,
+                           num_blocks=B * mbps + 1, max_blocks_per_seq=mbps,
+                           max_span_hint=span, max_query_len_hint=qlen, force_variant=fv,
+                           force_partitions=fp,
+                           kv_dtype=pa.PA_DTYPE_FP8_E4M3 if fp8 else pa.PA_DTYPE_BF16,
+                           k_scale=1.0 if fp8 else 0.0, v_scale=1.0 if fp8 else 0.0)
+        rc, info = pa.pa_plan(p, BS, 148, 2)
+        # pools past the TMA map's 32-bit rows run on the FMA kernel, which has
+        # no head_dim 256 and no FP8 path
+        fits = (B * mbps + 1) * hkv * BS <= 2 ** 31 - 1
+        fma = fv == pa.PA_VARIANT_FMA or not fits
+        if rc != pa.PA_OK:
+            assert rc == pa.PA_ERR_UNSUPPORTED and fma and (D == 256 or fp8), pa.pa_last_error()
+            continue
+        accepted += 1
+        P = info.max_partitions
+        assert info.partition_tokens % 64 == 0 and 1 <= P <= 16384
+        # the partitions cover the longest span plus the 64-token alignment of its start
+        assert P * info.partition_tokens >= span + 63 or P == 1
+        # the smem block-table slice caps a partition at its blocks plus two
+        cap = max(64, (1024 - 2) * BS // 64 * 64)
+        assert info.partition_tokens <= cap
+        if fp:  # "~n partitions": n, or one more for the start's alignment, unless capped
+            assert P <= fp + 1 or info.partition_tokens == cap
+        assert info.one_shot == (P == 1)
+        assert info.max_rows == grp * qlen
+        nslab = -(-info.max_rows // info.slab_rows)
+        assert (info.grid_x, info.grid_y, info.grid_z) == (P, hkv * nslab, B)
+        assert info.block_threads == 32 * (info.consumer_warps + 1)
+        assert info.smem_bytes <= 227 * 1024
+        if info.one_shot:
+            assert info.workspace_bytes == 0
+        else:
+            n = B * hkv * P * info.max_rows
+            assert info.workspace_bytes == align(n * 4) + align(n * D * 4)
+        assert info.variant == (pa.PA_VARIANT_FMA if fma else pa.PA_VARIANT_MMA)
+    assert accepted >= 400
