@@ -55,22 +55,37 @@ def _build(src_text, tmp_path, name):
 
 
 def _run_pins(so):
-    env = dict(os.environ, PA_ORACLE_LIB=so)
+    env = dict(os.environ, PA_ORACLE_LIB=so, OMP_NUM_THREADS="2")
     return subprocess.run([sys.executable, "-m", "pytest", PINS, "-x", "-q",
                            "-p", "no:cacheprovider"], cwd=ROOT, env=env,
                           capture_output=True, text=True, timeout=900)
 
 
-def test_control_build_passes_the_pins(tmp_path):
-    r = _run_pins(_build(open(SRC).read(), tmp_path, "control"))
+@pytest.fixture(scope="module")
+def pin_runs(tmp_path_factory):
+    """Every build's pin-suite run, the control's and each mutant's, run side
+    by side in separate processes (each starts its own interpreter)."""
+    from concurrent.futures import ThreadPoolExecutor
+    tmp = tmp_path_factory.mktemp("mutants")
+    src = open(SRC).read()
+    sources = {"control": src}
+    for name, (old, new) in MUTANTS.items():
+        assert src.count(old) == 1, f"mutation site of {name} not found once"
+        sources[name] = src.replace(old, new)
+    libs = {name: _build(text, tmp, name) for name, text in sources.items()}
+    workers = max(1, min(8, (os.cpu_count() or 2) // 2))
+    with ThreadPoolExecutor(max_workers=workers) as ex:
+        futures = {name: ex.submit(_run_pins, so) for name, so in libs.items()}
+        return {name: f.result() for name, f in futures.items()}
+
+
+def test_control_build_passes_the_pins(pin_runs):
+    r = pin_runs["control"]
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
 
 
 @pytest.mark.parametrize("name", list(MUTANTS))
-def test_pins_catch_a_planted_slip(name, tmp_path):
-    src = open(SRC).read()
-    old, new = MUTANTS[name]
-    assert src.count(old) == 1, f"mutation site of {name} not found once"
-    r = _run_pins(_build(src.replace(old, new), tmp_path, name))
+def test_pins_catch_a_planted_slip(name, pin_runs):
+    r = pin_runs[name]
     # exit code 1: tests ran and at least one failed (not a collection error)
     assert r.returncode == 1 and " failed" in r.stdout, r.stdout[-3000:] + r.stderr[-2000:]
