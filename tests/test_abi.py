@@ -382,3 +382,17 @@ def test_plan_invariants_on_random_params():
             assert info.workspace_bytes == align(n * 4) + align(n * D * 4)
         assert info.variant == (pa.PA_VARIANT_FMA if fma else pa.PA_VARIANT_MMA)
     assert accepted >= 400
+
+
+def test_import_fails_loudly_without_the_library(tmp_path):
+    # no fallback: a copy of the package without libpagedattn.so refuses to import
+    import shutil
+    import subprocess
+    import sys
+    pkg = os.path.dirname(pa.__file__)
+    dst = tmp_path / os.path.basename(pkg)
+    shutil.copytree(pkg, dst, ignore=shutil.ignore_patterns("*.so", "__pycache__"))
+    r = subprocess.run([sys.executable, "-c", f"import {dst.name}"], cwd=tmp_path,
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0
+    assert "ImportError" in r.stderr and "libpagedattn.so is missing" in r.stderr
