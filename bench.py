@@ -470,8 +470,8 @@ def oracle_sample_run(wl, rows, nthreads=0):
     """Runs the float64 oracle on the given rows of a workload (all heads);
     returns (seconds, kv+q+dst bytes of the sample, threads used)."""
     import oracle
-    from tests.parity_helpers import subproblem
-    pr, _ = subproblem(wl, rows)
+    sub, _ = wl.subset(rows)
+    pr = oracle.problem_from_workload(sub)
     sub_l = pr.query_lens.tolist()
     kv = 0
     for j, b in enumerate(sorted(set(rows))):

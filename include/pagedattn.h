@@ -70,7 +70,7 @@ extern "C" {
 #define PA_ERR_CUDA 4         /* a CUDA runtime call failed */
 
 /* Device status bits (pa_device_status). */
-#define PA_DEV_TIMEOUT 1u     /* a pipeline wait gave up after ~1 s */
+#define PA_DEV_TIMEOUT 1u     /* a bounded wait gave up (~1 s, or the wait_limit_cycles knob) */
 #define PA_DEV_BAD_ROW 2u     /* queryLens[b] > seqLens[b], negative length or window */
 #define PA_DEV_BAD_BLOCK 4u   /* a block-table entry outside [0, num_blocks) */
 #define PA_DEV_HINT 8u        /* a row longer than max_span_hint / max_query_len_hint */
@@ -141,6 +141,15 @@ typedef struct pa_params {
      * schedule's in the last bits (the stages' grouping depends on timing),
      * and it measures slower on the named workloads, so it is opt-in. */
     int schedule;
+    /* Test knobs of the one wait on other CTAs, the work-list merge's wait
+     * for its unit's arrivals (0 = off, the default).  wait_limit_cycles > 0
+     * replaces that wait's ~1 s limit (SM clock cycles); merge_target_extra
+     * > 0 raises the arrival count it waits for, so the count is never met:
+     * the wait gives up at the limit, the kernel returns, PA_DEV_TIMEOUT is
+     * set and the unit's dst rows are left unwritten.  The waits for the
+     * kernels' own bulk copies keep their fixed limit. */
+    long long wait_limit_cycles;
+    int merge_target_extra;
 } pa_params;
 
 /* What the dispatcher chose for a call (pa_plan). */
@@ -294,7 +303,10 @@ size_t pa_host_workspace_size(const pa_params *params, int kvBlockSize, int wind
  * passes every input and output.
  *
  *  - The first call on a device looks up the array's device address with
- *    that device current; make it before any stream capture.
+ *    that device current; make it before any stream capture.  A reset device
+ *    (cudaDeviceReset) has a new context and a new array: the first call
+ *    after the reset looks the address up again, so make that one before
+ *    any capture as well.
  *  - All calls on a device share the array: calls whose kernels overlap on
  *    the GPU race.  Nothing in it needs to start at zero; each call reads
  *    only partials it wrote itself.

@@ -148,6 +148,26 @@ class Problem:
         return int(self.query_lens.sum())
 
 
+def problem_from_workload(wl) -> Problem:
+    """A Problem holding host copies of a workload's buffers (any object with
+    the attributes of ``paged_kv_cache_474_b200.workloads.Workload``; its
+    tensors may live on any device).  bf16 tensors become their uint16 bit
+    patterns, FP8 code tensors stay uint8.  Marshalling only."""
+    import torch
+
+    def bits(t):
+        t = t.detach().contiguous().cpu()
+        if t.dtype == torch.uint8:
+            return t.numpy()
+        return t.view(torch.int16).numpy().view(np.uint16)
+
+    return Problem(bits(wl.q), bits(wl.k_cache), bits(wl.v_cache),
+                   wl.block_tables.cpu().numpy(), wl.seq_lens.cpu().numpy(),
+                   wl.query_lens.cpu().numpy(), wl.scale, wl.window,
+                   None if wl.windows is None else wl.windows.cpu().numpy(),
+                   k_scale=wl.k_scale, v_scale=wl.v_scale, q_scale=wl.q_scale)
+
+
 def decode(pr: Problem, parts: int = 0, nthreads: int = 0) -> np.ndarray:
     """All outputs, float64 [sum(query_lens), H_q, D].  parts=0: direct form;
     parts>0: split-K with that many partitions per row and a log-sum-exp merge."""

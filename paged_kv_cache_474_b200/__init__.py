@@ -63,6 +63,8 @@ class pa_params(ctypes.Structure):
         ("k_scale", ctypes.c_float),
         ("v_scale", ctypes.c_float),
         ("schedule", ctypes.c_int),
+        ("wait_limit_cycles", ctypes.c_longlong),
+        ("merge_target_extra", ctypes.c_int),
     ]
 
 

@@ -6,6 +6,7 @@
 """
 from __future__ import annotations
 
+import glob
 import os
 import subprocess
 import sys
@@ -15,7 +16,6 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libpagedattn.so")
 SOURCES = ["pa_kernels.cu", "pa_api.cu", "pa_noalloc.cu"]
-HEADERS = ["pa_device.cuh", "pa_kernels.cuh", "pa_span.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -27,7 +27,9 @@ def nvcc() -> str:
 
 
 def _inputs():
-    files = [os.path.join(CSRC, f) for f in SOURCES + HEADERS]
+    # every source and header under csrc/ (a header added later is covered too)
+    files = [os.path.join(CSRC, f) for f in SOURCES]
+    files += sorted(glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(CSRC, "*.h")))
     files.append(os.path.join(ROOT, "include", "pagedattn.h"))
     files.append(os.path.abspath(__file__))
     return files

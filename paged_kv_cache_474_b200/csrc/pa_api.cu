@@ -107,6 +107,8 @@ int check_params(const pa_params* p, int bs) {
   if (p->max_span_hint < 0 || p->max_query_len_hint < 0)
     return fail(PA_ERR_ARG, "hints must be >= 0");
   if (p->force_partitions < 0) return fail(PA_ERR_ARG, "force_partitions must be >= 0");
+  if (p->wait_limit_cycles < 0 || p->merge_target_extra < 0)
+    return fail(PA_ERR_ARG, "wait_limit_cycles and merge_target_extra must be >= 0");
   if (p->schedule != PA_SCHED_STATIC && p->schedule != PA_SCHED_WORKLIST)
     return fail(PA_ERR_ARG, "unknown schedule %d", p->schedule);
   if (p->force_variant != PA_VARIANT_AUTO && p->force_variant != PA_VARIANT_FMA &&
@@ -174,16 +176,16 @@ int make_plan(const pa_params* p, int bs, int span, int qlen, int num_sms, int c
   // Variant: the tensor-core kernel puts the KV tokens on the MMA's M axis
   // and the unit's rows on N (8 per tile), so it serves every row count; on
   // B200 it beats the CUDA-core FMA kernel even at 4 rows (GQA group 4 in an
-  // 8-wide tile: 122 vs 181 us on the GQA decode workload), because one
-  // m16n8k16 replaces ~40 FMA-path instructions per token.  The FMA kernel
-  // stays for pools whose row count exceeds the TMA map's 32-bit
-  // coordinates, and on request.
+  // 8-wide tile), because one m16n8k16 replaces ~40 FMA-path instructions per
+  // token and the FMA kernel becomes issue-bound.  The FMA kernel stays for
+  // pools whose row count exceeds the TMA map's 32-bit coordinates, and on
+  // request.
   //
   // The tensor-memory kernel (FP8 caches, head_dim 128) runs on request: it
   // feeds the e4m3 codes to tcgen05 straight from shared memory, but its
-  // softmax warps (one token per thread, eight per SM) are latency-bound and
-  // it trails the mma.sync kernel on the named workloads (GQA decode FP8:
-  // 97 vs 75 us).
+  // softmax warps (one token per thread) spend more issue slots per token
+  // than the conversions they save, so it trails the mma.sync kernel on the
+  // named workloads.
   const bool rows_fit_tma =
       (long long)p->num_blocks * p->num_kv_heads * bs <= (long long)INT32_MAX;
   const bool kv8 = p->kv_dtype == PA_DTYPE_FP8_E4M3;
@@ -531,6 +533,8 @@ int decode_impl(void* dst, const void* q, const void* kCache, const void* vCache
   a.max_rows = in.max_rows;
   a.slab_rows = in.slab_rows;
   a.num_slabs = in.grid_y / p->num_kv_heads;
+  a.wait_cycles = p->wait_limit_cycles > 0 ? p->wait_limit_cycles : pa::kWaitCycles;
+  a.wait_extra = p->merge_target_extra > 0 ? (unsigned int)p->merge_target_extra : 0u;
 
   const dim3 grid(in.grid_x, in.grid_y, in.grid_z);
   // One wave of window-free partitions (the few-units plan): a CTA's first

@@ -9,6 +9,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/pagedattn.h"
+#include "pa_kernels.cuh"
 #include "pa_span.h"
 
 namespace pa {
@@ -74,7 +75,6 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 // Bounded wait: spins on try_wait for at most ~kWaitCycles SM clocks (about a
 // second).  On timeout it records PA_DEV_TIMEOUT in the status word and
 // returns false; callers then stop consuming and leave the kernel cleanly.
-constexpr long long kWaitCycles = 2000000000LL;
 
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -135,14 +135,16 @@ __device__ __forceinline__ void epoch_arrive(unsigned long long* c, unsigned int
   atomicAdd(c, 1ull);
 }
 
-// Bounded wait (same limit as mbar_wait) for `target` arrivals of this epoch.
+// Bounded wait for `target` arrivals of this epoch on a counter other CTAs
+// bump: at most `limit` SM clocks (the call's wait_cycles, ~1 s unless a test
+// shortens it); on timeout PA_DEV_TIMEOUT is recorded and false returned.
 __device__ __forceinline__ bool epoch_wait(const unsigned long long* c, unsigned int epoch,
-                                           unsigned int target) {
+                                           unsigned int target, long long limit) {
   const long long t0 = clock64();
   while (true) {
     const unsigned long long v = ld_acquire_u64(c);
     if ((unsigned int)(v >> 32) == epoch && (unsigned int)v >= target) return true;
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > limit) {
       atomicOr(&g_pa_status, PA_DEV_TIMEOUT);
       return false;
     }

@@ -20,6 +20,7 @@
 #include <utility>
 
 #include <cuda.h>
+#include <cudaTypedefs.h>
 
 #include "pa_device.cuh"
 #include "pa_kernels.cuh"
@@ -542,7 +543,7 @@ __device__ __noinline__ void merge_unit_partials(const DecodeArgs& a, int b, int
   if (threadIdx.x == 0) {
     if (!touched) epoch_touch(cnt, a.epoch);
     atomicAdd(cnt, 1ull);
-    s_go = share && epoch_wait(cnt, a.epoch, (unsigned)nparts);
+    s_go = share && epoch_wait(cnt, a.epoch, (unsigned)nparts + a.wait_extra, a.wait_cycles);
     __threadfence();
   }
   __syncthreads();
@@ -1569,22 +1570,25 @@ __global__ void __launch_bounds__(256) pa_stage_kernel(const __grid_constant__ S
 }
 
 // Sets a kernel's dynamic-smem limit and asks for the largest shared-memory
-// carveout (so two CTAs fit per SM), once per (device, kernel, size).
+// carveout (so two CTAs fit per SM), once per (context, kernel, size): the
+// attributes belong to the context, so a context that replaced a reset one
+// gets them set again.
 cudaError_t ensure_smem_attrs(const void* kern, size_t smem) {
   static std::mutex mu;
-  static std::map<std::pair<int, const void*>, size_t> done;
+  static std::map<std::pair<unsigned long long, const void*>, size_t> done;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  const unsigned long long ctx = context_id();
   std::lock_guard<std::mutex> lock(mu);
-  auto it = done.find({dev, kern});
-  if (it != done.end() && it->second >= smem) return cudaSuccess;
+  auto it = done.find({ctx, kern});
+  if (ctx != 0 && it != done.end() && it->second >= smem) return cudaSuccess;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                            (int)cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
-  done[{dev, kern}] = smem;
+  if (ctx != 0) done[{ctx, kern}] = std::max(smem, it != done.end() ? it->second : (size_t)0);
   return cudaSuccess;
 }
 
@@ -1852,6 +1856,29 @@ cudaError_t launch_stage(const StageArgs& s, cudaStream_t stream) {
   if (s.n <= 0 || s.n > kMaxStageCopies || s.blocks <= 0) return cudaErrorInvalidValue;
   pa_stage_kernel<<<s.blocks, 256, 0, stream>>>(s);
   return cudaGetLastError();
+}
+
+unsigned long long context_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f);
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext c = nullptr;
+  if (get_current(&c) != CUDA_SUCCESS || c == nullptr) return 0;
+  unsigned long long id = 0;
+  if (get_id(c, &id) != CUDA_SUCCESS) return 0;
+  return id;
 }
 
 cudaError_t read_status(unsigned int* status, bool clear, cudaStream_t stream) {

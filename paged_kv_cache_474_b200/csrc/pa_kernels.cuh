@@ -12,6 +12,10 @@ namespace pa {
 
 constexpr int kStageTokens = 64;  // tokens per shared-memory pipeline stage
 constexpr int kMaxTableCache = 1024;  // block-table entries a CTA caches in smem
+// Limit of every bounded device wait, in SM clocks (about a second at the
+// B200's clocks); the work-list merge's wait takes pa_params.wait_limit_cycles
+// instead when that test knob is set.
+constexpr long long kWaitCycles = 2000000000LL;
 
 // Everything a decode launch needs; passed by value as a __grid_constant__.
 struct DecodeArgs {
@@ -48,6 +52,8 @@ struct DecodeArgs {
   unsigned int epoch;             // this call's tag for the counters below
   unsigned long long* stage_ctr;  // [B][grid.y] next stage to hand out
   unsigned long long* done;       // [B][grid.y] partials published
+  long long wait_cycles;          // limit of the merge's wait for arrivals (SM clocks)
+  unsigned int wait_extra;        // test knob: arrivals added to that wait's target
 };
 
 // Compile-time shape of a partition-kernel instance.
@@ -132,5 +138,11 @@ cudaError_t launch_stage(const StageArgs& s, cudaStream_t stream);
 
 // Reads (and optionally clears) the device status word.
 cudaError_t read_status(unsigned int* status, bool clear, cudaStream_t stream);
+
+// Unique id of the calling thread's current CUDA context, or 0 when there is
+// none yet (or the driver cannot say).  cudaDeviceReset replaces a device's
+// primary context, and kernel attributes and symbol addresses belong to the
+// context, so state cached across calls is keyed by this id.
+unsigned long long context_id();
 
 }  // namespace pa

@@ -12,7 +12,8 @@
 // Rules of use:
 //  - The first call on each device looks up the array's device address
 //    (cudaGetSymbolAddress, with that device current); make that first call
-//    before any stream capture.
+//    before any stream capture.  After cudaDeviceReset the first call in the
+//    new context looks it up again (the reset reloads the module).
 //  - Every call on a device shares the one array, so calls whose kernels
 //    overlap on the GPU (different streams, no ordering between them) race.
 //  - Nothing in the array has to start at zero: each call reads only the
@@ -26,6 +27,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/pagedattn.h"
+#include "pa_kernels.cuh"
 
 // The scratch array (file scope, internal linkage).
 static __device__ __align__(256) unsigned char g_noalloc_scratch[PA_NOALLOC_SCRATCH_BYTES];
@@ -34,20 +36,25 @@ namespace {
 
 constexpr int kMaxDevices = 128;
 
-// Device address of g_noalloc_scratch on the current device, looked up once
-// per device with that device current.  In host code the array's name is only
-// a host-side stand-in, so the kernels are given this address instead.
+// Device address of g_noalloc_scratch on the current device.  In host code
+// the array's name is only a host-side stand-in, so the kernels are given
+// this address instead.  It is looked up with the device current, once per
+// device and CUDA context: cudaDeviceReset replaces the device's context and
+// reloads the library's module, which moves the array, so a call made in a
+// new context looks the address up again.
 int scratch_address(void** out) {
   static std::mutex mu;
   static void* addr[kMaxDevices] = {};
+  static unsigned long long ctx_of[kMaxDevices] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
     fprintf(stderr, "pa_decode_noalloc: cannot read the current device\n");
     return PA_ERR_CUDA;
   }
+  const unsigned long long ctx = pa::context_id();
   std::lock_guard<std::mutex> lock(mu);
-  if (!addr[dev]) {
+  if (!addr[dev] || ctx == 0 || ctx != ctx_of[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || !p) {
@@ -56,6 +63,7 @@ int scratch_address(void** out) {
       return PA_ERR_CUDA;
     }
     addr[dev] = p;
+    ctx_of[dev] = pa::context_id();  // the lookup itself may have created the context
   }
   *out = addr[dev];
   return PA_OK;

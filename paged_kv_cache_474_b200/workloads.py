@@ -123,6 +123,39 @@ class Workload:
              else [self.window] * len(s))
         return s, l, w
 
+    def subset(self, rows):
+        """The given batch rows as a workload of their own, on the CPU: their
+        q rows, a compact pool holding only the blocks their tables reach
+        (tables renumbered to match, unused slots 0), their lengths and
+        windows; scales unchanged.  Data movement only.  Returns (workload,
+        row_map) with row_map[original row] = its index in the subset."""
+        rows = sorted(set(int(r) for r in rows))
+        S, L, _ = self.host_lists()
+        bs = self.block_size
+        tables = self.block_tables.cpu()
+        qoff = np.concatenate([[0], np.cumsum(L)]).astype(np.int64)
+        phys, new_tables = [], []
+        for b in rows:
+            nb = (S[b] + bs - 1) // bs
+            new_tables.append(list(range(len(phys), len(phys) + nb)))
+            phys.extend(tables[b, :nb].tolist())
+        mb = max(1, max(len(t) for t in new_tables))
+        tab = torch.zeros((len(rows), mb), dtype=torch.int32)
+        for j, t in enumerate(new_tables):
+            tab[j, :len(t)] = torch.tensor(t, dtype=torch.int32)
+        idx = torch.tensor(phys, dtype=torch.long, device=self.k_cache.device)
+        sub = dataclasses.replace(
+            self,
+            q=torch.cat([self.q[qoff[b]:qoff[b + 1]] for b in rows]).cpu(),
+            k_cache=self.k_cache.index_select(0, idx).cpu(),
+            v_cache=self.v_cache.index_select(0, idx).cpu(),
+            block_tables=tab,
+            seq_lens=torch.tensor([S[b] for b in rows], dtype=torch.int32),
+            query_lens=torch.tensor([L[b] for b in rows], dtype=torch.int32),
+            windows=(None if self.windows is None
+                     else self.windows.cpu()[torch.tensor(rows, dtype=torch.long)].clone()))
+        return sub, {b: j for j, b in enumerate(rows)}
+
 
 def bf16_bits(t: torch.Tensor) -> np.ndarray:
     """Host numpy view of a cache or q tensor's bit patterns: uint16 for bf16,

@@ -2,6 +2,7 @@
  * libpagedattn (no GPU needed).  tests/test_abi.py compiles it with
  * -std=c11 -pedantic -Werror, links it against the library, runs it and
  * compares its output with the same calls made through the Python binding. */
+#include <stddef.h>
 #include <stdio.h>
 #include <string.h>
 
@@ -43,5 +44,28 @@ int main(void)
     const int rc = pa_plan(&p, 16, 148, 2, &info);
     printf("refused %d %d\n", rc, (int)(strlen(pa_last_error()) > 0));
     printf("version %s\n", pa_version());
+    /* the structs' layout, field by field, for the binding's ctypes mirror */
+#define FIELD(T, f) printf("offset " #T "." #f " %zu\n", offsetof(T, f))
+    FIELD(pa_params, batch); FIELD(pa_params, num_q_heads); FIELD(pa_params, num_kv_heads);
+    FIELD(pa_params, head_dim); FIELD(pa_params, num_blocks);
+    FIELD(pa_params, max_blocks_per_seq); FIELD(pa_params, max_span_hint);
+    FIELD(pa_params, max_query_len_hint); FIELD(pa_params, windows);
+    FIELD(pa_params, workspace); FIELD(pa_params, workspace_bytes);
+    FIELD(pa_params, force_variant); FIELD(pa_params, force_partitions);
+    FIELD(pa_params, profile_events); FIELD(pa_params, q_dtype); FIELD(pa_params, kv_dtype);
+    FIELD(pa_params, q_scale); FIELD(pa_params, k_scale); FIELD(pa_params, v_scale);
+    FIELD(pa_params, schedule); FIELD(pa_params, wait_limit_cycles);
+    FIELD(pa_params, merge_target_extra);
+    FIELD(pa_plan_info, variant); FIELD(pa_plan_info, partition_tokens);
+    FIELD(pa_plan_info, max_partitions); FIELD(pa_plan_info, one_shot);
+    FIELD(pa_plan_info, max_rows); FIELD(pa_plan_info, slab_rows);
+    FIELD(pa_plan_info, consumer_warps); FIELD(pa_plan_info, stages);
+    FIELD(pa_plan_info, grid_x); FIELD(pa_plan_info, grid_y); FIELD(pa_plan_info, grid_z);
+    FIELD(pa_plan_info, block_threads); FIELD(pa_plan_info, smem_bytes);
+    FIELD(pa_plan_info, workspace_bytes); FIELD(pa_plan_info, num_sms);
+    FIELD(pa_plan_info, ctas_per_sm); FIELD(pa_plan_info, worklist);
+#undef FIELD
+    printf("sizeof pa_params %zu\n", sizeof(pa_params));
+    printf("sizeof pa_plan_info %zu\n", sizeof(pa_plan_info));
     return 0;
 }

@@ -8,7 +8,7 @@ import numpy as np
 import torch
 
 import oracle
-from paged_kv_cache_474_b200.workloads import Workload, bf16_bits, make_workload
+from paged_kv_cache_474_b200.workloads import Workload, make_workload
 
 ATOL = 2e-2
 RTOL = 2e-2
@@ -16,12 +16,7 @@ RTOL = 2e-2
 
 def problem(wl: Workload) -> oracle.Problem:
     """Whole workload as an oracle problem (host copies of every buffer)."""
-    return oracle.Problem(
-        bf16_bits(wl.q), bf16_bits(wl.k_cache), bf16_bits(wl.v_cache),
-        wl.block_tables.cpu().numpy(), wl.seq_lens.cpu().numpy(),
-        wl.query_lens.cpu().numpy(), wl.scale, wl.window,
-        None if wl.windows is None else wl.windows.cpu().numpy(),
-        k_scale=wl.k_scale, v_scale=wl.v_scale, q_scale=wl.q_scale)
+    return oracle.problem_from_workload(wl)
 
 
 def subproblem(wl: Workload, rows):
@@ -29,35 +24,8 @@ def subproblem(wl: Workload, rows):
     blocks their tables reach (gathered into a compact pool, tables
     remapped), lengths and windows.  Returns (problem, row_map) where row_map
     maps an original row to its index in the sub-problem."""
-    rows = sorted(set(int(r) for r in rows))
-    S = wl.seq_lens.cpu().tolist()
-    L = wl.query_lens.cpu().tolist()
-    W = wl.windows.cpu().tolist() if wl.windows is not None else None
-    bs = wl.block_size
-    tables = wl.block_tables.cpu()
-    qoff = np.concatenate([[0], np.cumsum(L)]).astype(np.int64)
-    phys = []
-    new_tables = []
-    for b in rows:
-        nb = (S[b] + bs - 1) // bs
-        ids = tables[b, :nb].tolist()
-        new_tables.append(list(range(len(phys), len(phys) + nb)))
-        phys.extend(ids)
-    mb = max(len(t) for t in new_tables)
-    tab = np.zeros((len(rows), mb), dtype=np.int32)
-    for j, t in enumerate(new_tables):
-        tab[j, :len(t)] = t
-    idx = torch.tensor(phys, dtype=torch.long, device=wl.k_cache.device)
-    kc = bf16_bits(wl.k_cache.index_select(0, idx))
-    vc = bf16_bits(wl.v_cache.index_select(0, idx))
-    qs = torch.cat([wl.q[qoff[b]:qoff[b + 1]] for b in rows])
-    pr = oracle.Problem(bf16_bits(qs), kc, vc, tab,
-                        np.array([S[b] for b in rows], dtype=np.int32),
-                        np.array([L[b] for b in rows], dtype=np.int32),
-                        wl.scale, wl.window,
-                        None if W is None else np.array([W[b] for b in rows], dtype=np.int32),
-                        k_scale=wl.k_scale, v_scale=wl.v_scale, q_scale=wl.q_scale)
-    return pr, {b: j for j, b in enumerate(rows)}
+    sub, rmap = wl.subset(rows)
+    return oracle.problem_from_workload(sub), rmap
 
 
 def token_offsets(wl: Workload):

@@ -1,6 +1,7 @@
 """CPU checks of the C ABI: the library loads, exports every symbol the header
 declares, validates arguments on the host, and plans partitions the way the
 dispatcher promises.  No call here launches GPU work."""
+import ctypes
 import os
 import re
 
@@ -313,7 +314,21 @@ def test_header_is_plain_c_and_matches_the_binding(tmp_path):
                     os.path.join(ROOT, "tests", "c_abi_check.c"), "-o", str(exe),
                     "-L", libdir, "-lpagedattn", f"-Wl,-rpath,{libdir}"], check=True)
     out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout
-    lines = dict(line.split(" ", 1) for line in out.strip().splitlines())
+    # every field of both structs sits where the binding's ctypes mirror puts it
+    nfield = 0
+    for line in out.strip().splitlines():
+        kind, rest = line.split(" ", 1)
+        if kind == "offset":
+            name, off = rest.split()
+            struct, field = name.split(".")
+            assert getattr(getattr(pa, struct), field).offset == int(off), name
+            nfield += 1
+        elif kind == "sizeof":
+            struct, size = rest.split()
+            assert ctypes.sizeof(getattr(pa, struct)) == int(size), struct
+    assert nfield == len(pa.pa_params._fields_) + len(pa.pa_plan_info._fields_)
+    lines = dict(line.split(" ", 1) for line in out.strip().splitlines()
+                 if line.split(" ", 1)[0] not in ("offset", "sizeof"))
     S, L, W = [300, 40, 7], [5, 1, 3], [16, 100, 2]
     span, qlen = pa.pa_extents_host(S, L, windows=W)
     assert lines["extents"] == f"{span} {qlen}"

@@ -474,3 +474,41 @@ def test_work_list_full_size_long_context_sampled():
     out = pa.decode(wl, schedule=pa.PA_SCHED_WORKLIST)
     torch.cuda.synchronize()
     check_sampled(wl, out, sample_queries(wl, 32, seed=77), "work list long context")
+
+
+@pytest.mark.parametrize("limit", [20_000, 2_000_000])
+def test_work_list_merge_wait_gives_up_and_the_next_call_is_correct(limit):
+    # The work-list merge waits for its unit's arrivals on a counter other
+    # CTAs bump; the wait is bounded.  The test knob raises the target by one
+    # so it is never met: every merging CTA gives up after `limit` SM clocks
+    # (~10 us or ~1 ms), the kernel returns, the status word says
+    # PA_DEV_TIMEOUT, and no dst element is written (the single row needs
+    # many partitions, so nothing takes the one-shot path).  The next normal
+    # call on the same workspace, with stale counters left behind, is exact.
+    wl = _wl_case("long")
+    d = dev(wl)
+    p = pa.params_for(d, schedule=pa.PA_SCHED_WORKLIST)
+    _, info = pa.pa_plan(p, wl.block_size)
+    assert info.worklist and info.max_partitions > 1
+    ws = pa.alloc_workspace(p, wl.block_size)
+    p.workspace, p.workspace_bytes = ws.data_ptr(), ws.numel()
+    p.wait_limit_cycles = limit
+    p.merge_target_extra = 1
+    out = torch.full(d.q.shape, float("nan"), dtype=torch.bfloat16, device="cuda:0")
+    assert _raw_decode(d, p, out) == pa.PA_OK, pa.pa_last_error()
+    torch.cuda.synchronize()
+    assert pa.pa_device_status(clear=True) == pa.PA_DEV_TIMEOUT
+    assert torch.isnan(out.float()).all()
+    p.wait_limit_cycles = 0
+    p.merge_target_extra = 0
+    for _ in range(2):
+        out = torch.full(d.q.shape, float("nan"), dtype=torch.bfloat16, device="cuda:0")
+        assert _raw_decode(d, p, out) == pa.PA_OK, pa.pa_last_error()
+        check_full(wl, out, "work list after a timed-out call")
+
+
+def test_wait_knobs_must_not_be_negative():
+    d = dev(_wl_case("long"))
+    p = pa.params_for(d, schedule=pa.PA_SCHED_WORKLIST)
+    p.wait_limit_cycles = -1
+    assert pa.pa_plan(p, 16)[0] == pa.PA_ERR_ARG

@@ -84,3 +84,31 @@ def test_fp8_caches_are_scaled_e4m3_codes_of_the_values():
     assert torch.all((codes - ref).abs()[big] <= ref.abs()[big] * 2.0 ** -4 + 1e-12)
     assert torch.isfinite(codes).all()
     assert not np.any(np.isin(q8.k_cache.numpy(), [0x7F, 0xFF]))  # no NaN codes
+
+
+@pytest.mark.parametrize("kv_dtype", ["bf16", "fp8_e4m3"])
+def test_row_subset_keeps_each_rows_problem(kv_dtype):
+    # Workload.subset gathers some rows into a compact pool with renumbered
+    # tables (the parity tests and the bench's oracle leg use it on the large
+    # workloads).  The oracle's outputs for those rows must not change at
+    # all, and the gathered blocks must be exactly the ones the rows use.
+    import oracle
+    wl = make_workload(seq_lens=[70, 5, 33, 128, 17], query_lens=[2, 1, 0, 3, 1],
+                       num_q_heads=6, num_kv_heads=2, head_dim=32, block_size=16,
+                       windows=[0, 3, 9, 40, 0], seed=5, spare_blocks=3, kv_dtype=kv_dtype)
+    full = oracle.decode(oracle.problem_from_workload(wl))
+    L = wl.query_lens.tolist()
+    qoff = np.concatenate([[0], np.cumsum(L)])
+    for rows in ([3], [0, 3], [4, 1, 2], [0, 1, 2, 3, 4]):
+        sub, rmap = wl.subset(rows)
+        assert sorted(rmap) == sorted(set(rows)) and sub.k_scale == wl.k_scale
+        nb = [(s + 15) // 16 for s in sub.seq_lens.tolist()]
+        assert sub.num_blocks == sum(nb)
+        for b, j in rmap.items():
+            used = wl.block_tables[b, :nb[j]].long()
+            assert torch.equal(sub.k_cache[sub.block_tables[j, :nb[j]].long()], wl.k_cache[used])
+            assert torch.equal(sub.v_cache[sub.block_tables[j, :nb[j]].long()], wl.v_cache[used])
+        got = oracle.decode(oracle.problem_from_workload(sub))
+        sl = np.concatenate([[0], np.cumsum(sub.query_lens.tolist())])
+        for b, j in rmap.items():
+            assert np.array_equal(got[sl[j]:sl[j + 1]], full[qoff[b]:qoff[b + 1]])
