@@ -33,6 +33,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "paged-attn decode µs/call and KV HBM GB/s (% of B200 peak) per config"
+VARIANTS = {"auto": 0, "fma": 1, "mma": 2, "tc": 3}   # pa_params.force_variant values
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -174,11 +175,11 @@ def run_ours(args, rank, world, local_rank):
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
     stream = torch.cuda.current_stream()
-    wl = config_workload(args.config, device=device, kv_dtype=args.kv_dtype)
+    wl = config_workload(args.config, device=device, kv_dtype=args.kv_dtype, rows=args.rows)
     kv_bytes, qo_bytes = algorithmic_bytes(wl)
     call_bytes = kv_bytes + qo_bytes
 
-    p = pa.params_for(wl)
+    p = pa.params_for(wl, force_variant=VARIANTS[args.variant])
     ws = pa.alloc_workspace(p, wl.block_size, device=device)
     if ws is not None:
         p.workspace, p.workspace_bytes = ws.data_ptr(), ws.numel()
@@ -252,6 +253,10 @@ def run_ours(args, rank, world, local_rank):
     peak, peak_kind = measured_hbm_peak()
     achieved = call_bytes / (kern_avg_ms * 1e-3) / 1e9
     title = CONFIG_TITLES[args.config] + ("" if args.kv_dtype == "bf16" else ", FP8 e4m3 KV")
+    if args.rows is not None:
+        title += f", first {wl.batch} rows"
+    if args.variant != "auto":
+        title += f", {args.variant} variant forced"
     traffic = traffic_from_profiles(kernel_source_hash(), title)
 
     # end to end through the host-buffer entry point
@@ -283,8 +288,9 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "peak_source": peak_kind,
-                     "kernel": ("pa_partition_mma_kernel" if plan.variant == pa.PA_VARIANT_MMA
-                                else "pa_partition_fma_kernel"),
+                     "kernel": {pa.PA_VARIANT_MMA: "pa_partition_mma_kernel",
+                                pa.PA_VARIANT_TC: "pa_partition_tc_kernel"}.get(
+                                    plan.variant, "pa_partition_fma_kernel"),
                      "kernel_us": round(kern_avg_ms * 1e3, 2),
                      "kernel_timing": "CUDA events the library records around the partition "
                                       "kernel, averaged over the timed steps re-run",
@@ -561,6 +567,10 @@ def main():
     ap.add_argument("--config", type=int, default=2)
     ap.add_argument("--kv-dtype", choices=["bf16", "fp8_e4m3"], default="bf16",
                     help="KV cache element type of the timed workload (FP8: per-tensor scaled e4m3)")
+    ap.add_argument("--variant", choices=sorted(VARIANTS), default="auto",
+                    help="kernel variant of the timed workload (profiling; auto = the dispatcher's)")
+    ap.add_argument("--rows", type=int, default=None,
+                    help="keep only the first rows of the workload (a reduced case for profiling)")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the per-config table and the CPU baseline")
     args = ap.parse_args()

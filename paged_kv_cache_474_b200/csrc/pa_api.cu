@@ -53,6 +53,7 @@ constexpr int TS = pa::kStageTokens;
 constexpr int kMinPartTokens = 256;
 constexpr int kManyUnitsMinTokens = 2048;
 constexpr int kManyUnitsMaxTokens = 4096;
+constexpr int kPrefetchStages = 2;  // stages a one-wave CTA prefetches before its wait
 constexpr unsigned long long kStageMaxBlocks = 512;  // CTAs per staging copy (256 threads each)
 
 bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
@@ -544,6 +545,13 @@ int decode_impl(void* dst, const void* q, const void* kCache, const void* vCache
                        window == 0 &&
                        (long long)in.grid_x * in.grid_y * in.grid_z <=
                            (long long)in.num_sms * in.ctas_per_sm;
+  // Before their grid-dependency wait, these CTAs prefetch their first
+  // stages into L2: in a decode loop the previous call's tail (its reduce,
+  // the handoff) would otherwise leave HBM idle.  Two stages measured best on
+  // the long single-group workload; three or more lost again (the prefetches
+  // compete with the previous call's last loads).
+  a.prefetch_stages = a.spec_first_stage ? kPrefetchStages : 0;
+  a.prefetch_first = 0;
   cudaEvent_t ev0 = nullptr, ev1 = nullptr;
   if (p->profile_events) {
     ev0 = static_cast<cudaEvent_t>(p->profile_events[0]);

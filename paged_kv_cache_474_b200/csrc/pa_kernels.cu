@@ -688,6 +688,31 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
   // another after this point before the main loops, so the copy warp's wait
   // for its table entries never holds up the compute warps' prologue.
   __syncthreads();
+  if (warp == 1 && a.prefetch_stages > 0) {
+    // L2 prefetch of the partition's first stages before the grid-dependency
+    // wait, by a compute warp (they only wait for staged data after it; the
+    // copy warp's path to its first copy stays as short as without it).  In a one-wave grid of window-free rows a partition starts at
+    // part * part_tokens whatever the lengths, so only its block-table
+    // entries are needed; the previous kernel may still rewrite them, so they
+    // are read with relaxed loads and steer nothing but these prefetches
+    // (clamped into the pool: every box lies inside the tensor map).  The
+    // copies proper re-read the table after the wait and find the boxes in
+    // L2 when nothing changed.
+    const int c0 = part * a.part_tokens + a.prefetch_first * TS;
+    const int br = min(a.block_size, TS);
+    const int ntok = min(min(a.prefetch_stages * TS, a.part_tokens - a.prefetch_first * TS),
+                         a.max_blocks_per_seq * a.block_size - c0);
+    const int nitem = 2 * (max(ntok, 0) / br);
+    const int32_t* tb = a.block_tables + (size_t)b * a.max_blocks_per_seq;
+    for (int i = lane; i < nitem; i += 32) {
+      const int t = c0 + (i >> 1) * br;
+      const int jj = t >> a.block_shift;
+      const int phys = min(max(ld_relaxed_s32(tb + jj), 0), a.num_blocks - 1);
+      tma_prefetch_3d((i & 1) ? static_cast<const void*>(&tmv) : static_cast<const void*>(&tmk), 0,
+                      (phys * a.num_kv_heads + kvh) * a.block_size + (t - (jj << a.block_shift)),
+                      0);
+    }
+  }
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
   const int S = a.seq_lens[b];
@@ -1362,31 +1387,40 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
 // dst = sum_p w_p O_p / sum_p w_p.  Partials are normalised, so the weights
 // carry each partition's softmax mass.
 //
-// One CTA per (row, kv head, batch row) and DSPLIT-th of head_dim, in one
-// pass over the partials: a partial's slice is DC/4 float4, so LPP lanes
-// share a partial and a warp reads 32/LPP partials per load; each lane loads
-// lse_p with its O_p slice (BATCH partials in flight) and keeps a running
-// (max, sum, weighted sum), merged across the lanes of a slice and then
-// across warps with the same rescale.  Rows with hundreds of partials split
-// head_dim over several CTAs so more SMs pull partials from L2.  Launched
-// with programmatic stream serialization: it is scheduled while the partition
-// kernel drains.  The lengths, windows and the row's q offset are read before
-// griddepcontrol.wait: they are inputs of the call, which the partition
-// kernel reads too, and it triggers this launch only after its own
+// One CTA per (row, kv head, batch row) and DSPLIT-th of head_dim.  A
+// partial's slice of DC dims is LPP = DC/4 lanes (one float4 each), so a warp
+// covers PPW = 32/LPP partials per load; the CTA's warps share the partials
+// so that a lane holds at most two of them per round, and its loads are
+// issued together before it merges them: one L2 round trip, whatever the
+// register allocator makes of the code.  (A deeper per-lane batch of eight
+// was compiled into a few dependent rounds at ~52 registers and took ~3.5 us
+// for the 293 partials of the long single-group workload; this takes one.)
+// Lanes keep a running (max, sum, weighted sum); lanes of a warp, then the
+// warps (through shared memory, merged as a tree by warp 0), combine with the
+// same rescale.  Rows with hundreds of partials split head_dim over more CTAs
+// so that 32 warps suffice and more SMs pull partials from L2.
+//
+// Launched with programmatic stream serialization: it is scheduled while the
+// partition kernel drains.  The lengths, windows and the row's q offset are
+// read before griddepcontrol.wait: they are inputs of the call, which the
+// partition kernel reads too, and it triggers this launch only after its own
 // griddepcontrol.wait, so whatever wrote them has completed.  Only the
-// partials are read after the wait: one trip to L2 once the partition grid
-// is done.
+// partials are read after the wait.
 // ---------------------------------------------------------------------------
 template <int D, int DSPLIT>
-__global__ void __launch_bounds__(512) pa_reduce_kernel(const __grid_constant__ DecodeArgs a) {
+__global__ void __launch_bounds__(1024) pa_reduce_kernel(const __grid_constant__ DecodeArgs a) {
   constexpr int DC = D / DSPLIT;  // dims per CTA
   constexpr int LPP = DC / 4;     // lanes per partial slice (one float4 each)
   constexpr int PPW = 32 / LPP;   // partials per warp load
-  constexpr int BATCH = 8;        // partials in flight per lane
-  __shared__ float s_m[16], s_z[16];
-  __shared__ float4 s_o[16][LPP];
+  static_assert(LPP >= 1 && LPP <= 32, "a partial's slice must fit a warp");
+  __shared__ float s_m[32][LPP], s_z[32][LPP];
+  __shared__ float4 s_o[32][LPP];
   __shared__ int s_qoff;
 
+  // The next call's partition kernel may launch now: its CTAs take the SMs
+  // the partition grid leaves, set up and prefetch while this grid works,
+  // and wait for its completion before reading any input.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int rr = blockIdx.x / DSPLIT, ch = blockIdx.x - (blockIdx.x / DSPLIT) * DSPLIT;
   const int kvh = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -1414,17 +1448,18 @@ __global__ void __launch_bounds__(512) pa_reduce_kernel(const __grid_constant__ 
   const size_t pst4 = (size_t)a.max_rows * D / 4;  // float4 stride between partials
   const int step = nw * PPW;
   LseAcc acc{kNegInf, 0.f, make_float4(0.f, 0.f, 0.f, 0.f)};
-  for (int p0 = warp * PPW + sub; p0 < nparts; p0 += BATCH * step) {
-    float l[BATCH];
-    float4 o[BATCH];
-#pragma unroll
-    for (int u = 0; u < BATCH; ++u) {
-      const int p = p0 + u * step;
-      l[u] = p < nparts ? lse[(size_t)p * a.max_rows] : kNegInf;
-      o[u] = p < nparts ? ob[(size_t)p * pst4] : make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int p0 = warp * PPW + sub; p0 < nparts; p0 += 2 * step) {
+    const int p1 = p0 + step;
+    const float l0 = lse[(size_t)p0 * a.max_rows];
+    const float4 o0 = ob[(size_t)p0 * pst4];
+    float l1 = kNegInf;
+    float4 o1 = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (p1 < nparts) {
+      l1 = lse[(size_t)p1 * a.max_rows];
+      o1 = ob[(size_t)p1 * pst4];
     }
-#pragma unroll
-    for (int u = 0; u < BATCH; ++u) lse_merge(acc, l[u], 1.f, o[u]);
+    lse_merge(acc, l0, 1.f, o0);
+    lse_merge(acc, l1, 1.f, o1);
   }
   // lanes holding the same dims (c4) in other slices of the warp
 #pragma unroll
@@ -1440,24 +1475,37 @@ __global__ void __launch_bounds__(512) pa_reduce_kernel(const __grid_constant__ 
   }
   if (sub == 0) {
     s_o[warp][c4] = acc.o;
-    if (c4 == 0) {
-      s_m[warp] = acc.m;
-      s_z[warp] = acc.z;
-    }
+    s_m[warp][c4] = acc.m;
+    s_z[warp][c4] = acc.z;
   }
   __syncthreads();
-  if (warp == 0 && lane < LPP) {
+  if (warp == 0) {
+    // warps' results as a tree: lane (g, c4) folds warps g, g + PPW, ...,
+    // then the PPW groups of each c4 combine by shuffles
     LseAcc t{kNegInf, 0.f, make_float4(0.f, 0.f, 0.f, 0.f)};
-    for (int i = 0; i < nw; ++i) lse_merge(t, s_m[i], s_z[i], s_o[i][lane]);
-    const float inv = t.z > 0.f ? 1.f / t.z : 0.f;
-    const int i = rr / a.group, j = rr - (rr / a.group) * a.group;
-    __nv_bfloat16* dp = a.dst +
-                        ((size_t)(s_qoff + i) * a.num_q_heads + (size_t)kvh * a.group + j) * D +
-                        ch * DC + lane * 4;
-    // one 8-byte store per lane: a warp writes whole 32-byte sectors (and
-    // whole write requests when dst is mapped host memory)
-    *reinterpret_cast<uint2*>(dp) = make_uint2(pack_bf16x2(t.o.x * inv, t.o.y * inv),
-                                               pack_bf16x2(t.o.z * inv, t.o.w * inv));
+    for (int i = sub; i < nw; i += PPW) lse_merge(t, s_m[i][c4], s_z[i][c4], s_o[i][c4]);
+#pragma unroll
+    for (int off = LPP; off < 32; off <<= 1) {
+      const float m2 = __shfl_xor_sync(FULL, t.m, off);
+      const float z2 = __shfl_xor_sync(FULL, t.z, off);
+      float4 o2;
+      o2.x = __shfl_xor_sync(FULL, t.o.x, off);
+      o2.y = __shfl_xor_sync(FULL, t.o.y, off);
+      o2.z = __shfl_xor_sync(FULL, t.o.z, off);
+      o2.w = __shfl_xor_sync(FULL, t.o.w, off);
+      lse_merge(t, m2, z2, o2);
+    }
+    if (sub == 0) {
+      const float inv = t.z > 0.f ? 1.f / t.z : 0.f;
+      const int i = rr / a.group, j = rr - (rr / a.group) * a.group;
+      __nv_bfloat16* dp = a.dst +
+                          ((size_t)(s_qoff + i) * a.num_q_heads + (size_t)kvh * a.group + j) * D +
+                          ch * DC + c4 * 4;
+      // one 8-byte store per lane: a warp writes whole 32-byte sectors (and
+      // whole write requests when dst is mapped host memory)
+      *reinterpret_cast<uint2*>(dp) = make_uint2(pack_bf16x2(t.o.x * inv, t.o.y * inv),
+                                                 pack_bf16x2(t.o.z * inv, t.o.w * inv));
+    }
   }
 }
 
@@ -1810,8 +1858,14 @@ cudaError_t launch_reduce_t(const DecodeArgs& a, cudaStream_t stream) {
   constexpr int PPW = 32 / (D / DSPLIT / 4);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.max_rows * DSPLIT, a.num_kv_heads, a.batch);
-  // warps so that each lane has about one batch of eight loads, 1 to 16
-  const int nw = max(1, min(16, (a.max_parts + PPW * 8 - 1) / (PPW * 8)));
+  // Warps per CTA, 1 to 32.  Few CTAs (one partition grid's worth of units
+  // is small): latency decides, so each lane takes at most two partials and
+  // all of them are in flight at once.  Many CTAs (the large-block MTP
+  // workload: 16K of them, 16 partials each): they hide each other's
+  // latency, so eight partials per lane (four rounds) keep the grid small.
+  const long long ctas = (long long)cfg.gridDim.x * cfg.gridDim.y * cfg.gridDim.z;
+  const int per_lane = ctas <= 1024 ? 2 : 8;
+  const int nw = max(1, min(32, (a.max_parts + per_lane * PPW - 1) / (per_lane * PPW)));
   cfg.blockDim = dim3(32 * nw);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
@@ -1824,16 +1878,24 @@ cudaError_t launch_reduce_t(const DecodeArgs& a, cudaStream_t stream) {
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
+// head_dim split of the reduce: the smallest of 1, 2, 4, ... (the first that
+// gives a partial's slice <= 32 lanes) at which 32 warps, two partials per
+// lane, cover the partials (only rows with more than 64 partials split).
+template <int D>
+cudaError_t launch_reduce_d(const DecodeArgs& a, cudaStream_t stream) {
+  auto fits = [&](int dsplit) { return 2 * 32 * (32 / (D / dsplit / 4)) >= a.max_parts; };
+  if constexpr (D <= 128)
+    if (fits(1)) return launch_reduce_t<D, 1>(a, stream);
+  if (fits(2)) return launch_reduce_t<D, 2>(a, stream);
+  if (fits(4)) return launch_reduce_t<D, 4>(a, stream);
+  if (fits(8)) return launch_reduce_t<D, 8>(a, stream);
+  return launch_reduce_t<D, 16>(a, stream);  // beyond this, lanes take more rounds
+}
+
 cudaError_t launch_reduce(const DecodeArgs& a, cudaStream_t stream) {
-  // Rows with many partials split head_dim over several CTAs (32 dims each);
-  // a CTA covers at most 128 dims (one float4 per lane).
-  const bool split = a.max_parts >= 64;
-  if (a.head_dim == 128)
-    return split ? launch_reduce_t<128, 4>(a, stream) : launch_reduce_t<128, 1>(a, stream);
-  if (a.head_dim == 64)
-    return split ? launch_reduce_t<64, 2>(a, stream) : launch_reduce_t<64, 1>(a, stream);
-  if (a.head_dim == 256)
-    return split ? launch_reduce_t<256, 8>(a, stream) : launch_reduce_t<256, 2>(a, stream);
+  if (a.head_dim == 128) return launch_reduce_d<128>(a, stream);
+  if (a.head_dim == 64) return launch_reduce_d<64>(a, stream);
+  if (a.head_dim == 256) return launch_reduce_d<256>(a, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -45,6 +45,11 @@ struct DecodeArgs {
   // stage before the lengths arrive (the longest rows fill the grid, so few
   // of those copies are for partitions past a row's end).
   int spec_first_stage;
+  // Stages of its partition each CTA prefetches into L2 before the
+  // grid-dependency wait (0: none), for the same one-wave grids of window-free
+  // rows: while the previous kernel drains, HBM would otherwise idle.
+  int prefetch_stages;
+  int prefetch_first;  // first stage of the partition it prefetches
   // Work-list schedule (tensor-core kernel, one-wave cooperative grid): a
   // unit's CTAs claim its 64-token stages from a counter and merge their own
   // partials instead of a reduce kernel.

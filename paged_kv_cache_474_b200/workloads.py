@@ -291,11 +291,17 @@ _SHAPES = {
 
 
 def config_workload(cfg: int, device="cpu", window: Optional[int] = None,
-                    kv_dtype: str = "bf16", q_dtype: str = "bf16") -> Workload:
+                    kv_dtype: str = "bf16", q_dtype: str = "bf16",
+                    rows: Optional[int] = None) -> Workload:
     """One of the five named workloads.  ``window`` overrides the scalar window
     (the tiny workload is run at window 0 and window 8); kv_dtype="fp8_e4m3"
-    quantises its caches to per-tensor-scaled FP8."""
+    quantises its caches to per-tensor-scaled FP8.  ``rows`` keeps only the
+    first rows of the batch (their lengths and windows unchanged; the pool
+    then holds only their blocks), a reduced case for profiling."""
     s, l, w, ws = config_lengths(cfg)
+    if rows is not None:
+        s, l = s[:rows], l[:rows]
+        ws = None if ws is None else ws[:rows]
     if window is not None:
         w = int(window)
     return make_workload(seq_lens=s, query_lens=l, window=w, windows=ws,
