@@ -552,6 +552,11 @@ int decode_impl(void* dst, const void* q, const void* kCache, const void* vCache
   // compete with the previous call's last loads).
   a.prefetch_stages = a.spec_first_stage ? kPrefetchStages : 0;
   a.prefetch_first = 0;
+  // FP8 caches, units of at most 8 rows: the compute warps take the stages in
+  // two pairs, two chunks at a time (measured a little faster on the GQA
+  // decode and long single-group workloads with FP8 caches).
+  a.pair_chunks = in.variant == PA_VARIANT_MMA && p->kv_dtype == PA_DTYPE_FP8_E4M3 &&
+                  in.max_rows <= 8 && !in.worklist;
   cudaEvent_t ev0 = nullptr, ev1 = nullptr;
   if (p->profile_events) {
     ev0 = static_cast<cudaEvent_t>(p->profile_events[0]);

@@ -650,6 +650,9 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
   using T = MmaTraits<D, F8>;
   using C = MmaCombine<D, NCW, N8>;
   constexpr int RT = C::RT;
+  // paired chunk processing (see the compute loop): FP8 caches, one n-tile,
+  // an even ring depth, four compute warps, the static schedule
+  constexpr bool PAIRABLE = F8 && N8 == 1 && NSTAGE % 2 == 0 && NCW == 4 && !WL;
   static_assert(C::BYTES <= NSTAGE * T::STAGE_BYTES, "combine area must fit in the ring");
 
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -677,9 +680,12 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
     if constexpr (WL) s_dtouch = 0;
     prefetch_tensormap(&tmk);
     prefetch_tensormap(&tmv);
+    // empty: one arrival per compute warp that consumes the stage (paired
+    // mode: two of them)
+    const uint32_t consumers = (PAIRABLE && a.pair_chunks) ? 2u : (uint32_t)NCW;
     for (int s = 0; s < NSTAGE; ++s) {
-      mbar_init(smem_u32(&bars[s]), 1);              // full: copy-warp arrival + tx bytes
-      mbar_init(smem_u32(&bars[NSTAGE + s]), NCW);   // empty: one arrival per compute warp
+      mbar_init(smem_u32(&bars[s]), 1);                   // full: copy-warp arrival + tx bytes
+      mbar_init(smem_u32(&bars[NSTAGE + s]), consumers);  // empty
     }
     fence_mbar_init();
   }
@@ -1112,8 +1118,220 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
 #pragma unroll
     for (int n = 0; n < N8; ++n) m_r[n][0] = m_r[n][1] = kNegInf, l_r[n][0] = l_r[n][1] = 0.f;
 
+    // Chunks of 16 tokens, NCH at a time: the scores of all NCH chunks, one
+    // online-softmax update over them, then their PV products.  With NCH = 2
+    // a warp carries two independent MMA chains through each phase.
+    auto process = [&](auto nch_c, int ch_first, int ch_step, int c0, uint32_t Ks, uint32_t Vs,
+                       bool all_valid, bool boundary) {
+      constexpr int NCH = decltype(nch_c)::value;
+      // S^T = K Q^T; a single chunk with one n-tile uses two accumulator sets
+      // (even / odd d steps) to halve the dependent MMA chain.
+      constexpr int NACC = (NCH == 1 && N8 == 1) ? 2 : 1;
+      int tbs[NCH];
+      uint32_t cbs[NCH];
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) {
+        tbs[c] = (ch_first + c * ch_step) * 16;
+        // the chunk's 16 tokens lie in one box (BR >= 16)
+        cbs[c] = (uint32_t)((tbs[c] >> brs) * box_bytes + (tbs[c] & (BR - 1)) * T::BOXW);
+      }
+      float sc[NCH][NACC][N8][4];
+#pragma unroll
+      for (int c = 0; c < NCH; ++c)
+#pragma unroll
+        for (int u = 0; u < NACC; ++u)
+#pragma unroll
+          for (int n = 0; n < N8; ++n)
+            sc[c][u][n][0] = sc[c][u][n][1] = sc[c][u][n][2] = sc[c][u][n][3] = 0.f;
+      if constexpr (F8) {
+        // one x4 = tokens 0-7 / 8-15 of chunks 2kp, 2kp+1: two k-steps
+#pragma unroll
+        for (int kp = 0; kp < T::KSTEPS / 2; ++kp) {
+#pragma unroll
+          for (int c = 0; c < NCH; ++c) {
+            uint32_t r[4];
+            ldsm_x4(Ks + cbs[c] + box_step_off<T::BOXW>(kp, kofs, half), r[0], r[1], r[2], r[3]);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              uint32_t ka[4];
+              e4m3x4_to_f16x2x2(r[2 * h], ka[0], ka[2]);
+              e4m3x4_to_f16x2x2(r[2 * h + 1], ka[1], ka[3]);
+              const int ks = 2 * kp + h;
+#pragma unroll
+              for (int n = 0; n < N8; ++n)
+                mma_f16_16816(sc[c][ks % NACC][n], ka, qb[ks][n][0], qb[ks][n][1]);
+            }
+          }
+        }
+      } else {
+#pragma unroll
+        for (int ks = 0; ks < T::KSTEPS; ++ks) {
+#pragma unroll
+          for (int c = 0; c < NCH; ++c) {
+            uint32_t ka[4];
+            ldsm_x4(Ks + cbs[c] + box_step_off<T::BOXW>(ks, kofs, half), ka[0], ka[1], ka[2],
+                    ka[3]);
+#pragma unroll
+            for (int n = 0; n < N8; ++n)
+              mma_bf16_16816(sc[c][ks % NACC][n], ka, qb[ks][n][0], qb[ks][n][1]);
+          }
+        }
+      }
+      // element e of n-tile n: token tb + quad + 8*(e>>1), row n*8 + 2*qi + (e&1)
+      float p[NCH][N8][4];
+      bool any_rescale = false;
+      float al[N8][2];
+#pragma unroll
+      for (int n = 0; n < N8; ++n) {
+        float v[NCH][4];
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float x = sc[c][0][n][e];
+            if constexpr (NACC == 2) x += sc[c][1][n][e];
+            v[c][e] = x * a.scale_log2;
+          }
+          if (!all_valid) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int t = c0 + tbs[c] + quad + ((e >> 1) << 3);
+              v[c][e] = (t >= lo_r[n][e & 1] && t < hi_r[n][e & 1]) ? v[c][e] : kNegInf;
+            }
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          float mx = fmaxf(v[0][j], v[0][j + 2]);
+#pragma unroll
+          for (int c = 1; c < NCH; ++c) mx = fmaxf(mx, fmaxf(v[c][j], v[c][j + 2]));
+          mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 4));
+          mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 8));
+          mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 16));
+          // The running maximum moves only when the chunks' maximum passes it
+          // by more than kLazyMax (log2 units): probabilities stay below
+          // 2^kLazyMax, and after the first chunks O is rarely rescaled.
+          const bool up = mx > m_r[n][j] + kLazyMax;  // m_r = -inf: any finite mx
+          const float mn = up ? mx : m_r[n][j];
+          const float mu = (mn == kNegInf) ? 0.f : mn;
+          al[n][j] = up ? ex2(m_r[n][j] - mu) : 1.f;  // first update: 2^-inf = 0 (O, l are 0)
+          any_rescale |= up;
+          m_r[n][j] = mn;
+          float ps = 0.f;
+#pragma unroll
+          for (int c = 0; c < NCH; ++c) {
+            p[c][n][j] = ex2(v[c][j] - mu);
+            p[c][n][j + 2] = ex2(v[c][j + 2] - mu);
+            ps += p[c][n][j] + p[c][n][j + 2];
+          }
+          l_r[n][j] = l_r[n][j] * al[n][j] + ps;
+        }
+      }
+      if (__any_sync(FULL, any_rescale)) {
+#pragma unroll
+        for (int md = 0; md < T::MD; ++md)
+#pragma unroll
+          for (int n = 0; n < N8; ++n) {
+            o[md][n][0] *= al[n][0];
+            o[md][n][1] *= al[n][1];
+            o[md][n][2] *= al[n][0];
+            o[md][n][3] *= al[n][1];
+          }
+      }
+      // P^T B fragments: the accumulator's 8x8 blocks transposed in registers.
+      uint32_t pb[NCH][N8][2];
+#pragma unroll
+      for (int c = 0; c < NCH; ++c)
+#pragma unroll
+        for (int n = 0; n < N8; ++n) {
+          if constexpr (F8) {
+            pb[c][n][0] = movmatrix_trans(pack_f16x2(p[c][n][0], p[c][n][1]));
+            pb[c][n][1] = movmatrix_trans(pack_f16x2(p[c][n][2], p[c][n][3]));
+          } else {
+            pb[c][n][0] = movmatrix_trans(pack_bf16x2(p[c][n][0], p[c][n][1]));
+            pb[c][n][1] = movmatrix_trans(pack_bf16x2(p[c][n][2], p[c][n][3]));
+          }
+        }
+      uint32_t mk_lo[NCH], mk_hi[NCH];
+#pragma unroll
+      for (int c = 0; c < NCH; ++c) {
+        mk_lo[c] = mk_hi[c] = 0xffffffffu;
+        if (boundary) {
+          const int t = c0 + tbs[c] + 2 * qi;
+          auto in = [&](int u) { return u >= ulo && u < p1; };
+          mk_lo[c] = (in(t) ? 0x0000ffffu : 0u) | (in(t + 1) ? 0xffff0000u : 0u);
+          mk_hi[c] = (in(t + 8) ? 0x0000ffffu : 0u) | (in(t + 9) ? 0xffff0000u : 0u);
+        }
+      }
+      // O^T += V^T P^T; the V lanes of tokens outside [ulo, p1) are zeroed
+      // only in stages that reach past those bounds (masked = true).
+      auto pv = [&](auto masked) {
+        constexpr bool MK = decltype(masked)::value;
+        if constexpr (F8) {
+          // one x4.trans = tokens 0-7 / 8-15 of chunks 2mp, 2mp+1: two M
+          // tiles; a register holds dims (2g, 2g+1) of tokens (2c, 2c+1),
+          // regrouped by dim before the conversion (masks act on f16 halves)
+#pragma unroll
+          for (int mp = 0; mp < T::MD / 2; ++mp) {
+#pragma unroll
+            for (int c = 0; c < NCH; ++c) {
+              uint32_t r[4];
+              ldsm_x4_t(Vs + cbs[c] + box_step_off<T::BOXW>(mp, vofs, half), r[0], r[1], r[2],
+                        r[3]);
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                uint32_t va[4];
+                e4m3x4_to_f16x2x2(__byte_perm(r[2 * h], 0, 0x3120), va[0], va[1]);
+                e4m3x4_to_f16x2x2(__byte_perm(r[2 * h + 1], 0, 0x3120), va[2], va[3]);
+                if constexpr (MK) {
+                  va[0] &= mk_lo[c];
+                  va[1] &= mk_lo[c];
+                  va[2] &= mk_hi[c];
+                  va[3] &= mk_hi[c];
+                }
+#pragma unroll
+                for (int n = 0; n < N8; ++n)
+                  mma_f16_16816(o[2 * mp + h][n], va, pb[c][n][0], pb[c][n][1]);
+              }
+            }
+          }
+        } else {
+#pragma unroll
+          for (int md = 0; md < T::MD; ++md) {
+#pragma unroll
+            for (int c = 0; c < NCH; ++c) {
+              uint32_t va[4];
+              ldsm_x4_t(Vs + cbs[c] + box_step_off<T::BOXW>(md, vofs, half), va[0], va[1],
+                        va[2], va[3]);
+              if constexpr (MK) {
+                va[0] &= mk_lo[c];
+                va[1] &= mk_lo[c];
+                va[2] &= mk_hi[c];
+                va[3] &= mk_hi[c];
+              }
+#pragma unroll
+              for (int n = 0; n < N8; ++n) mma_bf16_16816(o[md][n], va, pb[c][n][0], pb[c][n][1]);
+            }
+          }
+        }
+      };
+      if (boundary)
+        pv(std::true_type{});
+      else
+        pv(std::false_type{});
+    };
+
+    // Paired mode (FP8 caches, units of at most 8 rows, an even ring depth):
+    // warps 1-2 consume the even stages and warps 3-4 the odd ones, each warp
+    // two chunks of its stage at once, so each ring slot always serves the
+    // same two warps (a parity wait never skips one of its phases).  Every
+    // other case: every compute warp consumes every stage, its chunks one by
+    // one.
+    const bool paired = PAIRABLE && a.pair_chunks;
+    const int kfirst = paired ? (slice >> 1) : 0;
+    const int kstep = paired ? 2 : 1;
     const int kend = WL ? INT_MAX : nst;
-    for (int k = 0; k < kend; ++k) {
+    for (int k = kfirst; k < kend; k += kstep) {
       const int s = k % NSTAGE;
       const bool got = mbar_wait(smem_u32(&bars[s]), (k / NSTAGE) & 1);
       if (!__all_sync(FULL, got)) break;
@@ -1126,163 +1344,17 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
       const uint32_t Vs = Ks + T::KV_BYTES;
       const bool all_valid = (c0 >= lo_max) && (c0 + TS <= hi_min);
       const bool boundary = (c0 < ulo) || (c0 + TS > p1);
-
-      for (int ch = slice; ch < TS / 16; ch += nslice) {
-        const int tb = ch * 16;
-        // the chunk's 16 tokens lie in one box (BR >= 16)
-        const uint32_t cbase = (uint32_t)((tb >> brs) * box_bytes + (tb & (BR - 1)) * T::BOXW);
-        // S^T = K Q^T; with one n-tile, two accumulator sets (even / odd d
-        // steps) halve the dependent MMA chain.
-        constexpr int NACC = N8 == 1 ? 2 : 1;
-        float sc[2][N8][4];
-#pragma unroll
-        for (int u = 0; u < 2; ++u)
-#pragma unroll
-          for (int n = 0; n < N8; ++n) sc[u][n][0] = sc[u][n][1] = sc[u][n][2] = sc[u][n][3] = 0.f;
-        if constexpr (F8) {
-          // one x4 = tokens 0-7 / 8-15 of chunks 2kp, 2kp+1: two k-steps
-#pragma unroll
-          for (int kp = 0; kp < T::KSTEPS / 2; ++kp) {
-            uint32_t r[4];
-            ldsm_x4(Ks + cbase + box_step_off<T::BOXW>(kp, kofs, half), r[0], r[1], r[2], r[3]);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              uint32_t ka[4];
-              e4m3x4_to_f16x2x2(r[2 * h], ka[0], ka[2]);
-              e4m3x4_to_f16x2x2(r[2 * h + 1], ka[1], ka[3]);
-              const int ks = 2 * kp + h;
-#pragma unroll
-              for (int n = 0; n < N8; ++n)
-                mma_f16_16816(sc[ks % NACC][n], ka, qb[ks][n][0], qb[ks][n][1]);
-            }
-          }
+      if constexpr (PAIRABLE) {
+        if (paired) {
+          process(std::integral_constant<int, 2>{}, 2 * (slice & 1), 1, c0, Ks, Vs, all_valid,
+                  boundary);
         } else {
-#pragma unroll
-          for (int ks = 0; ks < T::KSTEPS; ++ks) {
-            uint32_t ka[4];
-            ldsm_x4(Ks + cbase + box_step_off<T::BOXW>(ks, kofs, half), ka[0], ka[1], ka[2],
-                    ka[3]);
-#pragma unroll
-            for (int n = 0; n < N8; ++n)
-              mma_bf16_16816(sc[ks % NACC][n], ka, qb[ks][n][0], qb[ks][n][1]);
-          }
+          for (int ch = slice; ch < TS / 16; ch += nslice)
+            process(std::integral_constant<int, 1>{}, ch, 0, c0, Ks, Vs, all_valid, boundary);
         }
-        // element e of n-tile n: token tb + quad + 8*(e>>1), row n*8 + 2*qi + (e&1)
-        float p[N8][4];
-        bool any_rescale = false;
-        float al[N8][2];
-#pragma unroll
-        for (int n = 0; n < N8; ++n) {
-          float v[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) v[e] = (sc[0][n][e] + sc[1][n][e]) * a.scale_log2;
-          if (!all_valid) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int t = c0 + tb + quad + ((e >> 1) << 3);
-              v[e] = (t >= lo_r[n][e & 1] && t < hi_r[n][e & 1]) ? v[e] : kNegInf;
-            }
-          }
-#pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            float mx = fmaxf(v[j], v[j + 2]);
-            mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 4));
-            mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 8));
-            mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, 16));
-            // The running maximum moves only when the chunk's maximum passes it
-            // by more than kLazyMax (log2 units): probabilities stay below
-            // 2^kLazyMax, and after the first chunks O is rarely rescaled.
-            const bool up = mx > m_r[n][j] + kLazyMax;  // m_r = -inf: any finite mx
-            const float mn = up ? mx : m_r[n][j];
-            const float mu = (mn == kNegInf) ? 0.f : mn;
-            al[n][j] = up ? ex2(m_r[n][j] - mu) : 1.f;  // first update: 2^-inf = 0 (O, l are 0)
-            any_rescale |= up;
-            m_r[n][j] = mn;
-            p[n][j] = ex2(v[j] - mu);
-            p[n][j + 2] = ex2(v[j + 2] - mu);
-            l_r[n][j] = l_r[n][j] * al[n][j] + (p[n][j] + p[n][j + 2]);
-          }
-        }
-        if (__any_sync(FULL, any_rescale)) {
-#pragma unroll
-          for (int md = 0; md < T::MD; ++md)
-#pragma unroll
-            for (int n = 0; n < N8; ++n) {
-              o[md][n][0] *= al[n][0];
-              o[md][n][1] *= al[n][1];
-              o[md][n][2] *= al[n][0];
-              o[md][n][3] *= al[n][1];
-            }
-        }
-        // P^T B fragments: the accumulator's 8x8 blocks transposed in registers.
-        uint32_t pb[N8][2];
-#pragma unroll
-        for (int n = 0; n < N8; ++n) {
-          if constexpr (F8) {
-            pb[n][0] = movmatrix_trans(pack_f16x2(p[n][0], p[n][1]));
-            pb[n][1] = movmatrix_trans(pack_f16x2(p[n][2], p[n][3]));
-          } else {
-            pb[n][0] = movmatrix_trans(pack_bf16x2(p[n][0], p[n][1]));
-            pb[n][1] = movmatrix_trans(pack_bf16x2(p[n][2], p[n][3]));
-          }
-        }
-        uint32_t mk_lo = 0xffffffffu, mk_hi = 0xffffffffu;
-        if (boundary) {
-          const int t = c0 + tb + 2 * qi;
-          auto in = [&](int u) { return u >= ulo && u < p1; };
-          mk_lo = (in(t) ? 0x0000ffffu : 0u) | (in(t + 1) ? 0xffff0000u : 0u);
-          mk_hi = (in(t + 8) ? 0x0000ffffu : 0u) | (in(t + 9) ? 0xffff0000u : 0u);
-        }
-        // O^T += V^T P^T; the V lanes of tokens outside [ulo, p1) are zeroed
-        // only in stages that reach past those bounds (masked = true).
-        auto pv = [&](auto masked) {
-          constexpr bool MK = decltype(masked)::value;
-          if constexpr (F8) {
-            // one x4.trans = tokens 0-7 / 8-15 of chunks 2mp, 2mp+1: two M
-            // tiles; a register holds dims (2g, 2g+1) of tokens (2c, 2c+1),
-            // regrouped by dim before the conversion (masks act on f16 halves)
-#pragma unroll
-            for (int mp = 0; mp < T::MD / 2; ++mp) {
-              uint32_t r[4];
-              ldsm_x4_t(Vs + cbase + box_step_off<T::BOXW>(mp, vofs, half), r[0], r[1], r[2],
-                        r[3]);
-#pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                uint32_t va[4];
-                e4m3x4_to_f16x2x2(__byte_perm(r[2 * h], 0, 0x3120), va[0], va[1]);
-                e4m3x4_to_f16x2x2(__byte_perm(r[2 * h + 1], 0, 0x3120), va[2], va[3]);
-                if constexpr (MK) {
-                  va[0] &= mk_lo;
-                  va[1] &= mk_lo;
-                  va[2] &= mk_hi;
-                  va[3] &= mk_hi;
-                }
-#pragma unroll
-                for (int n = 0; n < N8; ++n)
-                  mma_f16_16816(o[2 * mp + h][n], va, pb[n][0], pb[n][1]);
-              }
-            }
-          } else {
-#pragma unroll
-            for (int md = 0; md < T::MD; ++md) {
-              uint32_t va[4];
-              ldsm_x4_t(Vs + cbase + box_step_off<T::BOXW>(md, vofs, half), va[0], va[1],
-                        va[2], va[3]);
-              if constexpr (MK) {
-                va[0] &= mk_lo;
-                va[1] &= mk_lo;
-                va[2] &= mk_hi;
-                va[3] &= mk_hi;
-              }
-#pragma unroll
-              for (int n = 0; n < N8; ++n) mma_bf16_16816(o[md][n], va, pb[n][0], pb[n][1]);
-            }
-          }
-        };
-        if (boundary)
-          pv(std::true_type{});
-        else
-          pv(std::false_type{});
+      } else {
+        for (int ch = slice; ch < TS / 16; ch += nslice)
+          process(std::integral_constant<int, 1>{}, ch, 0, c0, Ks, Vs, all_valid, boundary);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars[NSTAGE + s]));

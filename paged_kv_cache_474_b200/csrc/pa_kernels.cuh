@@ -50,6 +50,9 @@ struct DecodeArgs {
   // rows: while the previous kernel drains, HBM would otherwise idle.
   int prefetch_stages;
   int prefetch_first;  // first stage of the partition it prefetches
+  // Tensor-core kernel with FP8 caches, units of at most 8 rows: the compute
+  // warps work in two pairs on alternating stages, two chunks at a time.
+  int pair_chunks;
   // Work-list schedule (tensor-core kernel, one-wave cooperative grid): a
   // unit's CTAs claim its 64-token stages from a counter and merge their own
   // partials instead of a reduce kernel.
