@@ -241,12 +241,32 @@ int make_plan(const pa_params* p, int bs, int span, int qlen, int num_sms, int c
     int rc = current_sms(&num_sms);
     if (rc) return rc;
   }
+  const bool caller_occupancy = ctas_per_sm > 0;
   if (ctas_per_sm <= 0) {
     ctas_per_sm = cached_occupancy(mma, pl.shape, smem_for(cap));
     if (ctas_per_sm <= 0)
       return fail(PA_ERR_CUDA, "occupancy query failed: %s", cudaGetErrorString(cudaGetLastError()));
   }
   const long long units = (long long)p->batch * p->num_kv_heads * nslab;
+  // FP8 caches, head_dim 128, units of one n-tile, a grid of few units (one
+  // balanced wave): a six-stage ring at two CTAs per SM instead of four
+  // stages at three.  Each CTA then has four stages in flight while its two
+  // warp pairs work on the other two, and the wave has fewer, longer
+  // partitions for the reduce to merge; measured on the long single-group
+  // workload, 21.5 -> 19.5 us per isolated call and 14.8 -> 13.9 us in
+  // back-to-back calls.  Grids of many units keep three CTAs per SM (the
+  // deeper ring lost there: 64.4 -> 72.2 us on GQA decode).
+  if (kv8 && !tc && variant == PA_VARIANT_MMA && p->head_dim == 128 && n8 == 1 &&
+      p->force_partitions <= 0 && !caller_occupancy) {
+    pa::KernelShape deep = pl.shape;
+    deep.stages = 6;
+    const int c6 =
+        cached_occupancy(true, deep, pa::mma_smem_bytes(p->head_dim, 1, 6, cap, bs));
+    if (c6 > 0 && units * 4 <= (long long)num_sms * c6) {
+      pl.shape = deep;
+      ctas_per_sm = c6;
+    }
+  }
   const long long slots = (long long)num_sms * ctas_per_sm;
 
   long long ptok;

@@ -1859,7 +1859,8 @@ size_t mma_smem_bytes(int head_dim, int elem_bytes, int stages, int part_tokens,
 
 // (head_dim, compute warps, stages, n-tiles, FP8 caches).  Rings: bf16 64,
 // 96 and 192 KB for head_dim 64, 128 and 256; FP8 64 KB (head_dim 64, 128:
-// three CTAs per SM fit at 128) and 96 KB (256: two CTAs per SM).
+// three CTAs per SM fit at 128) and 96 KB (256: two CTAs per SM; 128 with
+// six stages, for one-wave grids of single-tile units).
 #define PA_MMA_DISPATCH(CALL)                                                       \
   if (k.head_dim == 128 && k.consumer_warps == 4 && k.stages == 3 && k.n8 == 1 && !k.kv_fp8) \
     CALL(128, 4, 3, 1, false);                                                      \
@@ -1875,6 +1876,8 @@ size_t mma_smem_bytes(int head_dim, int elem_bytes, int stages, int part_tokens,
     CALL(128, 4, 4, 1, true);                                                       \
   if (k.head_dim == 128 && k.consumer_warps == 4 && k.stages == 4 && k.n8 == 2 && k.kv_fp8)  \
     CALL(128, 4, 4, 2, true);                                                       \
+  if (k.head_dim == 128 && k.consumer_warps == 4 && k.stages == 6 && k.n8 == 1 && k.kv_fp8)  \
+    CALL(128, 4, 6, 1, true);                                                       \
   if (k.head_dim == 64 && k.consumer_warps == 4 && k.stages == 8 && k.n8 == 1 && k.kv_fp8)   \
     CALL(64, 4, 8, 1, true);                                                        \
   if (k.head_dim == 64 && k.consumer_warps == 4 && k.stages == 8 && k.n8 == 2 && k.kv_fp8)   \
