@@ -1469,8 +1469,8 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
 // for the 293 partials of the long single-group workload; this takes one.)
 // Lanes keep a running (max, sum, weighted sum); lanes of a warp, then the
 // warps (through shared memory, merged as a tree by warp 0), combine with the
-// same rescale.  Rows with hundreds of partials split head_dim over more CTAs
-// so that 32 warps suffice and more SMs pull partials from L2.
+// same rescale.  Rows with many partials split head_dim over more CTAs so
+// that 16 warps suffice and more SMs pull partials from L2.
 //
 // Launched with programmatic stream serialization: it is scheduled while the
 // partition kernel drains.  The lengths, windows and the row's q offset are
@@ -1954,11 +1954,14 @@ cudaError_t launch_reduce_t(const DecodeArgs& a, cudaStream_t stream) {
 }
 
 // head_dim split of the reduce: the smallest of 1, 2, 4, ... (the first that
-// gives a partial's slice <= 32 lanes) at which 32 warps, two partials per
-// lane, cover the partials (only rows with more than 64 partials split).
+// gives a partial's slice <= 32 lanes) at which 16 warps, two partials per
+// lane, cover the partials (only rows with more than 32 partials split).
+// Measured on the long single-group workload (293 partials per row): 16 CTAs
+// per row of 10 warps each beat 8 of 19 warps by 0.7 us per call in
+// back-to-back calls (bf16 and FP8); 32 CTAs of 5 warps, or 4 of 32, lost.
 template <int D>
 cudaError_t launch_reduce_d(const DecodeArgs& a, cudaStream_t stream) {
-  auto fits = [&](int dsplit) { return 2 * 32 * (32 / (D / dsplit / 4)) >= a.max_parts; };
+  auto fits = [&](int dsplit) { return 2 * 16 * (32 / (D / dsplit / 4)) >= a.max_parts; };
   if constexpr (D <= 128)
     if (fits(1)) return launch_reduce_t<D, 1>(a, stream);
   if (fits(2)) return launch_reduce_t<D, 2>(a, stream);
