@@ -577,6 +577,10 @@ int decode_impl(void* dst, const void* q, const void* kCache, const void* vCache
   // decode and long single-group workloads with FP8 caches).
   a.pair_chunks = in.variant == PA_VARIANT_MMA && p->kv_dtype == PA_DTYPE_FP8_E4M3 &&
                   in.max_rows <= 8 && !in.worklist;
+  // Token rows per TMA box: a block, or a 64-token slice of a larger one; at
+  // most 32 when the paired compute warps refill their own halves (the
+  // four-stage FP8 ring), so that no box crosses a stage's halves.
+  a.box_rows = std::min(bs, (a.pair_chunks && pl.shape.stages <= 4) ? TS / 2 : TS);
   cudaEvent_t ev0 = nullptr, ev1 = nullptr;
   if (p->profile_events) {
     ev0 = static_cast<cudaEvent_t>(p->profile_events[0]);
@@ -587,7 +591,7 @@ int decode_impl(void* dst, const void* q, const void* kCache, const void* vCache
     if (in.variant == PA_VARIANT_MMA || in.variant == PA_VARIANT_TC) {
       CUtensorMap tk, tv;
       const long long rows = (long long)p->num_blocks * p->num_kv_heads * bs;
-      const int br = std::min(bs, TS);
+      const int br = in.variant == PA_VARIANT_TC ? std::min(bs, TS) : a.box_rows;
       const int eb = p->kv_dtype == PA_DTYPE_FP8_E4M3 ? 1 : 2;
       rc = kv_tensor_map(&tk, kCache, rows, p->head_dim, eb, br);
       if (!rc) rc = kv_tensor_map(&tv, vCache, rows, p->head_dim, eb, br);

@@ -653,6 +653,10 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
   // paired chunk processing (see the compute loop): FP8 caches, one n-tile,
   // an even ring depth, four compute warps, the static schedule
   constexpr bool PAIRABLE = F8 && N8 == 1 && NSTAGE % 2 == 0 && NCW == 4 && !WL;
+  // ... whose compute warps refill their own halves (rings of at most four
+  // stages: the six-stage ring serves one-wave grids, whose partitions need
+  // about one refill per CTA, and there the extra code cost 0.8 us per call)
+  constexpr bool SELFREF = PAIRABLE && NSTAGE <= 4;
   static_assert(C::BYTES <= NSTAGE * T::STAGE_BYTES, "combine area must fit in the ring");
 
   extern __shared__ __align__(128) uint8_t smem_raw[];
@@ -667,6 +671,11 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
   const int kvh = blockIdx.y % a.num_kv_heads;
   const int slab = blockIdx.y / a.num_kv_heads;
   const int part = blockIdx.x;
+  // Paired mode (see the compute loop): a compute warp owns one half (32
+  // tokens) of every other stage; with self-refill it also refills that half.
+  const bool paired = PAIRABLE && a.pair_chunks;
+  const bool selfref = SELFREF && a.pair_chunks;
+  const int BR = a.box_rows;  // token rows per TMA box (<= 32 with self-refill)
 
   __shared__ int s_qoff;
   __shared__ float s_fac[NCW][64], s_rowm[64], s_rowz[64];  // warp-merge factors (rows <= 64)
@@ -680,12 +689,13 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
     if constexpr (WL) s_dtouch = 0;
     prefetch_tensormap(&tmk);
     prefetch_tensormap(&tmv);
-    // empty: one arrival per compute warp that consumes the stage (paired
-    // mode: two of them)
-    const uint32_t consumers = (PAIRABLE && a.pair_chunks) ? 2u : (uint32_t)NCW;
+    // full: one arrival with the tx bytes per copy; empty: one arrival per
+    // compute warp that consumes the stage (paired mode: two).  Self-refill
+    // has no empty barriers: bars[NSTAGE + s] is the full barrier of slot s's
+    // second half.
     for (int s = 0; s < NSTAGE; ++s) {
-      mbar_init(smem_u32(&bars[s]), 1);                   // full: copy-warp arrival + tx bytes
-      mbar_init(smem_u32(&bars[NSTAGE + s]), consumers);  // empty
+      mbar_init(smem_u32(&bars[s]), 1);
+      mbar_init(smem_u32(&bars[NSTAGE + s]), selfref ? 1u : paired ? 2u : (uint32_t)NCW);
     }
     fence_mbar_init();
   }
@@ -705,7 +715,7 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
     // copies proper re-read the table after the wait and find the boxes in
     // L2 when nothing changed.
     const int c0 = part * a.part_tokens + a.prefetch_first * TS;
-    const int br = min(a.block_size, TS);
+    const int br = BR;
     const int ntok = min(min(a.prefetch_stages * TS, a.part_tokens - a.prefetch_first * TS),
                          a.max_blocks_per_seq * a.block_size - c0);
     const int nitem = 2 * (max(ntok, 0) / br);
@@ -742,32 +752,42 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
     const int c0 = part * a.part_tokens;
     if (a.spec_first_stage && c0 + TS <= a.max_blocks_per_seq * a.block_size) {
       __syncwarp();
-      const int br = min(a.block_size, TS);
-      const int nitem0 = (TS / br) * 2;
-      const uint32_t bb = (uint32_t)br * T::ROW_BYTES;
-      uint32_t dst = 0;
+      const int nitem0 = (TS / BR) * 2;
+      const uint32_t bb = (uint32_t)BR * T::ROW_BYTES;
+      uint32_t dst = 0, bar = smem_u32(&bars[0]);
       int y = 0, isv = 0;
       if (lane < nitem0) {
         const int jb = lane >> 1;
         isv = lane & 1;
-        const int bt0 = c0 + jb * br;
+        const int bt0 = c0 + jb * BR;
         const int jj = bt0 >> a.block_shift;
         const int phys = min(max(bt_s[jj - sj0], 0), a.num_blocks - 1);
         y = (phys * a.num_kv_heads + kvh) * a.block_size + (bt0 - (jj << a.block_shift));
         dst = isv * T::KV_BYTES + jb * bb;
+        if (selfref && jb * BR >= TS / 2) bar = smem_u32(&bars[NSTAGE]);
       }
-      if (lane == 0) mbar_arrive_expect_tx(smem_u32(&bars[0]), (uint32_t)nitem0 * bb);
+      if (lane == 0) {
+        if (selfref) {  // each half: its own barrier, half the items
+          mbar_arrive_expect_tx(smem_u32(&bars[0]), (uint32_t)(nitem0 / 2) * bb);
+          mbar_arrive_expect_tx(smem_u32(&bars[NSTAGE]), (uint32_t)(nitem0 / 2) * bb);
+        } else {
+          mbar_arrive_expect_tx(smem_u32(&bars[0]), (uint32_t)nitem0 * bb);
+        }
+      }
       __syncwarp();
       if (lane < nitem0)
         tma_load_3d_hint(smem_u32(smem) + dst,
                          isv ? static_cast<const void*>(&tmv) : static_cast<const void*>(&tmk), 0,
-                         y, 0, smem_u32(&bars[0]), l2_evict_first_policy());
+                         y, 0, bar, l2_evict_first_policy());
       spec0 = true;
     }
   }
   // A CTA that leaves with a speculative stage in flight first waits for it.
   auto leave = [&]() {
-    if (spec0 && lane == 0) mbar_wait(smem_u32(&bars[0]), 0);
+    if (spec0 && lane == 0) {
+      mbar_wait(smem_u32(&bars[0]), 0);
+      if (selfref) mbar_wait(smem_u32(&bars[NSTAGE]), 0);
+    }
   };
   if (L <= 0) {
     leave();
@@ -815,7 +835,6 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
   const int NRT = (Rs + RT - 1) / RT;  // row tiles in this slab
 
   // A box is BR token rows of one (block, kv head): [halves][BR rows][BOXW bytes].
-  const int BR = min(a.block_size, TS);
   const uint32_t box_bytes = (uint32_t)BR * T::ROW_BYTES;
   int qoff = 0;
 
@@ -935,16 +954,19 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
           }
         }
       }
-      const uint32_t nload = __popc(__ballot_sync(FULL, mine));
+      // self-refill: boxes of the stage's second half complete its own barrier
+      const bool hi = selfref && lane < nitem && (lane >> 1) * BR >= TS / 2;
+      const uint32_t all = __ballot_sync(FULL, mine), high = __ballot_sync(FULL, mine && hi);
       if (lane == 0) {
         if constexpr (WL) s_c0[s] = c0;
-        mbar_arrive_expect_tx(smem_u32(&bars[s]), nload * box_bytes);
+        mbar_arrive_expect_tx(smem_u32(&bars[s]), __popc(all & ~high) * box_bytes);
+        if (selfref) mbar_arrive_expect_tx(smem_u32(&bars[NSTAGE + s]), __popc(high) * box_bytes);
       }
       __syncwarp();
       if (mine)
         tma_load_3d_hint(smem_u32(smem) + dst,
                          isv ? static_cast<const void*>(&tmv) : static_cast<const void*>(&tmk), 0,
-                         y, 0, smem_u32(&bars[s]), kv_policy);
+                         y, 0, smem_u32(&bars[hi ? NSTAGE + s : s]), kv_policy);
       return true;
     };
     // Work list, after stage kk's copies: the next stage numbers, the claim
@@ -990,7 +1012,9 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
     int k = spec0 ? 1 : 0;
     bool ok = true;
     if constexpr (!WL) {
-      for (; k < nst; ++k)
+      // self-refill: the first ring's worth only; the compute warps refill
+      const int kcopy = selfref ? min(nst, NSTAGE) : nst;
+      for (; k < kcopy; ++k)
         if (!issue(k, p0 + k * TS, 0)) {
           ok = false;
           break;
@@ -1026,7 +1050,8 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
         mbar_arrive(smem_u32(&bars[s]));
       }
     }
-    if (lane == 0) {
+    // (self-refill: the compute warps wait for every stage this warp issued)
+    if (lane == 0 && !selfref) {
       for (int kk = max(0, issued - NSTAGE + (WL ? 1 : 0)); kk < issued; ++kk)
         mbar_wait(smem_u32(&bars[kk % NSTAGE]), (kk / NSTAGE) & 1);
     }
@@ -1040,7 +1065,7 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
     const int quad = lane >> 2, qi = lane & 3;
     qoff = row_token_offset(a.query_lens, b, lane);
     if (warp == 1 && lane == 0) s_qoff = qoff;  // for the copy warp's share of the merge
-    const int brs = a.block_shift < 6 ? a.block_shift : 6;  // log2(BR)
+    const int brs = 31 - __clz(BR);  // log2(BR)
     // lane parts of the ldmatrix row addresses (token row within the chunk,
     // 16-byte chunk parity) for K (A operand) and V (A operand, transposed)
     const int lt_k = (((lane >> 3) & 1) << 3) + (lane & 7), ck_k = lane >> 4;
@@ -1323,18 +1348,61 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
 
     // Paired mode (FP8 caches, units of at most 8 rows, an even ring depth):
     // warps 1-2 consume the even stages and warps 3-4 the odd ones, each warp
-    // two chunks of its stage at once, so each ring slot always serves the
-    // same two warps (a parity wait never skips one of its phases).  Every
-    // other case: every compute warp consumes every stage, its chunks one by
-    // one.
-    const bool paired = PAIRABLE && a.pair_chunks;
+    // two chunks (one 32-token half) of its stage at once, so each warp
+    // carries two MMA chains, and each ring slot always serves the same two
+    // warps (a parity wait never skips one of its phases).  With self-refill
+    // each warp also refills its own half of the slot with the stage NSTAGE
+    // ahead as soon as it has read it: the copy warp, whose 8 box requests per
+    // stage took ~600 cycles to issue, would otherwise sit between every
+    // release and the next copy.  Each half then has its own full barrier,
+    // waited for and re-armed by that one warp.  Every other case: every
+    // compute warp consumes every stage, its chunks one by one, and the copy
+    // warp refills the ring.
     const int kfirst = paired ? (slice >> 1) : 0;
     const int kstep = paired ? 2 : 1;
     const int kend = WL ? INT_MAX : nst;
+    const int hsel = slice & 1;  // paired mode: this warp's half of its stages
+    const uint64_t kv_policy_c = l2_evict_first_policy();
+    // Self-refill: copies this warp's half of stage kk into slot s (barrier fb).
+    auto refill = [&](int kk, int s, uint32_t fb) {
+      fence_proxy_async_smem();  // this warp's reads of the half, before the copies overwrite it
+      const int hs = p0 + kk * TS + hsel * (TS / 2);  // the half's first token
+      const int ta = max(hs, ulo), te = min(hs + TS / 2, p1);
+      const int nb = (TS / 2) / BR;  // boxes per half
+      bool mine = false;
+      uint32_t dst = 0;
+      int y = 0, isv = 0;
+      if (lane < 2 * nb) {
+        const int j = lane >> 1;
+        isv = lane & 1;
+        const int bt0 = hs + j * BR;
+        if (bt0 + BR > ta && bt0 < te) {
+          const int jj = bt0 >> a.block_shift;
+          const int phys = bt_s[jj - jb0];
+          if (phys >= 0) {
+            mine = true;
+            y = (phys * a.num_kv_heads + kvh) * a.block_size + (bt0 - (jj << a.block_shift));
+            dst = s * T::STAGE_BYTES + isv * T::KV_BYTES + (hsel * nb + j) * box_bytes;
+          }
+        }
+      }
+      const uint32_t nload = __popc(__ballot_sync(FULL, mine));
+      if (lane == 0) mbar_arrive_expect_tx(fb, nload * box_bytes);
+      __syncwarp();
+      if (mine)
+        tma_load_3d_hint(smem_u32(smem) + dst,
+                         isv ? static_cast<const void*>(&tmv) : static_cast<const void*>(&tmk), 0,
+                         y, 0, fb, kv_policy_c);
+    };
+    int kgave = -1;  // self-refill: the stage whose wait gave up
     for (int k = kfirst; k < kend; k += kstep) {
       const int s = k % NSTAGE;
-      const bool got = mbar_wait(smem_u32(&bars[s]), (k / NSTAGE) & 1);
-      if (!__all_sync(FULL, got)) break;
+      const uint32_t fb = smem_u32(&bars[(selfref && hsel) ? NSTAGE + s : s]);
+      const bool got = mbar_wait(fb, (k / NSTAGE) & 1);
+      if (!__all_sync(FULL, got)) {
+        kgave = k;
+        break;
+      }
       int c0 = p0 + k * TS;
       if constexpr (WL) {
         c0 = s_c0[s];
@@ -1357,7 +1425,18 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
           process(std::integral_constant<int, 1>{}, ch, 0, c0, Ks, Vs, all_valid, boundary);
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars[NSTAGE + s]));
+      if (selfref) {
+        if (k + NSTAGE < kend) refill(k + NSTAGE, s, fb);
+      } else if (lane == 0) {
+        mbar_arrive(smem_u32(&bars[NSTAGE + s]));
+      }
+    }
+    if (selfref && kgave >= 0 && lane == 0) {
+      // A wait gave up (the status is set): this warp's copies still in
+      // flight, the stage it waited for and the next one of its slots, land
+      // (bounded waits) before the CTA can leave.
+      for (int kk = kgave; kk < kend && kk <= kgave + 2; kk += 2)
+        mbar_wait(smem_u32(&bars[hsel ? NSTAGE + kk % NSTAGE : kk % NSTAGE]), (kk / NSTAGE) & 1);
     }
 
     named_bar_sync(1, NCW * 32);

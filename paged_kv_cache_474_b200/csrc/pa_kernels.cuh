@@ -50,6 +50,7 @@ struct DecodeArgs {
   // rows: while the previous kernel drains, HBM would otherwise idle.
   int prefetch_stages;
   int prefetch_first;  // first stage of the partition it prefetches
+  int box_rows;        // token rows per TMA box of the tensor-core kernel (<= 32 in paired mode)
   // Tensor-core kernel with FP8 caches, units of at most 8 rows: the compute
   // warps work in two pairs on alternating stages, two chunks at a time.
   int pair_chunks;
