@@ -303,3 +303,36 @@ def test_tensor_memory_kernel_full_size_sampled(cfg):
     out = pa.decode(wl, force_variant=TC)
     torch.cuda.synchronize()
     check_sampled(wl, out, sample_queries(wl, 32, seed=200 + cfg), f"cfg{cfg} tc full size")
+
+
+@pytest.mark.parametrize("block_size", [16, 32, 64, 256, 1024])
+@pytest.mark.parametrize("parts", [0, 3])
+def test_fp8_one_wave_and_self_refill_rings(block_size, parts):
+    # FP8 caches, units of at most 8 rows.  A one-wave grid (few units, the
+    # dispatcher's own partitions) runs the six-stage ring at two CTAs per SM,
+    # refilled by the copy warp; a forced partition count keeps the four-stage
+    # ring, whose compute warps refill their own half stages with boxes of at
+    # most 32 rows (slices of the larger blocks).
+    wl = make_workload(seq_lens=[1, 63, 64, 700, 2049, 5000], query_lens=[1, 1, 1, 2, 1, 2],
+                       num_q_heads=16, num_kv_heads=4, head_dim=128, block_size=block_size,
+                       seed=block_size + parts, kv_dtype=FP8)
+    d = dev(wl)
+    rc, info = pa.pa_plan(pa.params_for(d, force_partitions=parts), block_size)
+    assert rc == pa.PA_OK
+    assert info.stages == (6 if parts == 0 else 4)
+    out = pa.decode(d, force_partitions=parts)
+    check_full(wl, out, f"fp8 ring BS={block_size} parts={parts}")
+
+
+def test_fp8_self_refill_on_a_grid_of_many_units():
+    # many units (several waves of CTAs): the four-stage ring with self-refill
+    # chosen by the dispatcher itself, ragged rows, every element checked
+    g = np.random.default_rng(21)
+    S = g.integers(1, 3000, size=48).tolist()
+    wl = make_workload(seq_lens=S, query_lens=[1] * 48, num_q_heads=32, num_kv_heads=8,
+                       head_dim=128, block_size=16, seed=21, kv_dtype=FP8)
+    d = dev(wl)
+    rc, info = pa.pa_plan(pa.params_for(d), 16)
+    assert rc == pa.PA_OK and info.stages == 4
+    out = pa.decode(d)
+    check_full(wl, out, "fp8 self-refill, many units")
