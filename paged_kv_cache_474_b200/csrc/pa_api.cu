@@ -252,10 +252,9 @@ int make_plan(const pa_params* p, int bs, int span, int qlen, int num_sms, int c
   // balanced wave): a six-stage ring at two CTAs per SM instead of four
   // stages at three.  Each CTA then has four stages in flight while its two
   // warp pairs work on the other two, and the wave has fewer, longer
-  // partitions for the reduce to merge; measured on the long single-group
-  // workload, 21.5 -> 19.5 us per isolated call and 14.8 -> 13.9 us in
-  // back-to-back calls.  Grids of many units keep three CTAs per SM (the
-  // deeper ring lost there: 64.4 -> 72.2 us on GQA decode).
+  // partitions for the reduce to merge (faster on the long single-group
+  // workload).  Grids of many units keep three CTAs per SM: there the extra
+  // warps hide more latency than the deeper ring (it lost on GQA decode).
   if (kv8 && !tc && variant == PA_VARIANT_MMA && p->head_dim == 128 && n8 == 1 &&
       p->force_partitions <= 0 && !caller_occupancy) {
     pa::KernelShape deep = pl.shape;
@@ -573,8 +572,9 @@ int decode_impl(void* dst, const void* q, const void* kCache, const void* vCache
   a.prefetch_stages = a.spec_first_stage ? kPrefetchStages : 0;
   a.prefetch_first = 0;
   // FP8 caches, units of at most 8 rows: the compute warps take the stages in
-  // two pairs, two chunks at a time (measured a little faster on the GQA
-  // decode and long single-group workloads with FP8 caches).
+  // two pairs, two chunks at a time, and with the four-stage ring each warp
+  // refills its own half stages (measured faster on the GQA decode and long
+  // single-group workloads with FP8 caches).
   a.pair_chunks = in.variant == PA_VARIANT_MMA && p->kv_dtype == PA_DTYPE_FP8_E4M3 &&
                   in.max_rows <= 8 && !in.worklist;
   // Token rows per TMA box: a block, or a 64-token slice of a larger one; at

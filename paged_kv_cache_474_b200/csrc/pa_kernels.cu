@@ -655,7 +655,7 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
   constexpr bool PAIRABLE = F8 && N8 == 1 && NSTAGE % 2 == 0 && NCW == 4 && !WL;
   // ... whose compute warps refill their own halves (rings of at most four
   // stages: the six-stage ring serves one-wave grids, whose partitions need
-  // about one refill per CTA, and there the extra code cost 0.8 us per call)
+  // about one refill per CTA, so there the extra code only costs registers)
   constexpr bool SELFREF = PAIRABLE && NSTAGE <= 4;
   static_assert(C::BYTES <= NSTAGE * T::STAGE_BYTES, "combine area must fit in the ring");
 
@@ -1352,8 +1352,8 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
     // carries two MMA chains, and each ring slot always serves the same two
     // warps (a parity wait never skips one of its phases).  With self-refill
     // each warp also refills its own half of the slot with the stage NSTAGE
-    // ahead as soon as it has read it: the copy warp, whose 8 box requests per
-    // stage took ~600 cycles to issue, would otherwise sit between every
+    // ahead as soon as it has read it: the copy warp, which issues a stage's 8
+    // box requests one after another, would otherwise sit between every
     // release and the next copy.  Each half then has its own full barrier,
     // waited for and re-armed by that one warp.  Every other case: every
     // compute warp consumes every stage, its chunks one by one, and the copy
@@ -1544,8 +1544,8 @@ __global__ void __maxnreg__((N8 == 1 && D <= 128) ? 128 : 168)
 // so that a lane holds at most two of them per round, and its loads are
 // issued together before it merges them: one L2 round trip, whatever the
 // register allocator makes of the code.  (A deeper per-lane batch of eight
-// was compiled into a few dependent rounds at ~52 registers and took ~3.5 us
-// for the 293 partials of the long single-group workload; this takes one.)
+// was compiled into a few dependent rounds at a low register count: several
+// L2 round trips for the hundreds of partials of a long row; this takes one.)
 // Lanes keep a running (max, sum, weighted sum); lanes of a warp, then the
 // warps (through shared memory, merged as a tree by warp 0), combine with the
 // same rescale.  Rows with many partials split head_dim over more CTAs so
@@ -2034,10 +2034,10 @@ cudaError_t launch_reduce_t(const DecodeArgs& a, cudaStream_t stream) {
 
 // head_dim split of the reduce: the smallest of 1, 2, 4, ... (the first that
 // gives a partial's slice <= 32 lanes) at which 16 warps, two partials per
-// lane, cover the partials (only rows with more than 32 partials split).
-// Measured on the long single-group workload (293 partials per row): 16 CTAs
-// per row of 10 warps each beat 8 of 19 warps by 0.7 us per call in
-// back-to-back calls (bf16 and FP8); 32 CTAs of 5 warps, or 4 of 32, lost.
+// lane, cover the partials (only rows with more than 32 partials split):
+// more, smaller CTAs pull a long row's partials from L2 in parallel and fold
+// a shorter tree; far smaller ones (a lane per partial) load each partial's
+// lse once per lane and lost again.
 template <int D>
 cudaError_t launch_reduce_d(const DecodeArgs& a, cudaStream_t stream) {
   auto fits = [&](int dsplit) { return 2 * 16 * (32 / (D / dsplit / 4)) >= a.max_parts; };
