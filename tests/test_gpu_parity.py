@@ -512,3 +512,22 @@ def test_wait_knobs_must_not_be_negative():
     p = pa.params_for(d, schedule=pa.PA_SCHED_WORKLIST)
     p.wait_limit_cycles = -1
     assert pa.pa_plan(p, 16)[0] == pa.PA_ERR_ARG
+
+
+@pytest.mark.parametrize("head_dim", [64, 128, 256])
+@pytest.mark.parametrize("parts", [33, 65, 129, 300, 700, 1500])
+def test_reduce_splits_over_partial_counts(head_dim, parts):
+    # The reduce splits head_dim so that at most 16 warps, two partials per
+    # lane, cover a row's partials: forced partition counts of one 8-row unit
+    # (64-token partitions, a ragged last one) reach every split from one to
+    # sixteen CTAs per row and, past 512 partials, several rounds per lane.
+    S = parts * 64 - 5
+    wl = make_workload(seq_lens=[S], query_lens=[1], num_q_heads=8, num_kv_heads=1,
+                       head_dim=head_dim, block_size=64, seed=parts + head_dim)
+    d = dev(wl)
+    rc, info = pa.pa_plan(pa.params_for(d, force_partitions=parts), 64)
+    # 64-token partitions: the row has `parts` of them (the plan sizes for one
+    # more, the 64-token alignment of a span's start)
+    assert rc == pa.PA_OK and info.partition_tokens == 64
+    out = pa.decode(d, force_partitions=parts)
+    check_full(wl, out, f"reduce D={head_dim} parts={parts}")
