@@ -336,3 +336,42 @@ def test_fp8_self_refill_on_a_grid_of_many_units():
     assert rc == pa.PA_OK and info.stages == 4
     out = pa.decode(d)
     check_full(wl, out, "fp8 self-refill, many units")
+
+
+@pytest.mark.parametrize("block_size", [16, 64])
+def test_fp8_self_refill_never_reads_outside_spans(block_size):
+    # A grid of many units takes the four-stage ring whose compute warps pick
+    # and copy their own boxes.  NaN codes past each row's last token, before
+    # each window and in blocks no table reaches must not reach the outputs.
+    g = np.random.default_rng(23 + block_size)
+    B = 48
+    S = g.integers(1, 3000, size=B).tolist()
+    L = g.integers(1, 3, size=B).tolist()
+    W = [int(w) if g.random() < 0.6 else 0 for w in g.integers(1, 2500, size=B)]
+    L = [min(l, s) for l, s in zip(L, S)]
+    wl = make_workload(seq_lens=S, query_lens=L, num_q_heads=8, num_kv_heads=2, head_dim=128,
+                       block_size=block_size, windows=W, seed=23 + block_size, spare_blocks=2,
+                       extra_table_cols=3, kv_dtype=FP8)
+    ref = oracle.decode(problem(wl))
+    bs = block_size
+    for b in range(B):
+        nb = (S[b] + bs - 1) // bs
+        last = int(wl.block_tables[b, nb - 1])
+        wl.k_cache[last, :, S[b] - (nb - 1) * bs:] = NAN_CODE
+        wl.v_cache[last, :, S[b] - (nb - 1) * bs:] = NAN_CODE
+        first = max(0, S[b] - L[b] + 1 - W[b]) if W[b] > 0 else 0
+        for t in range(first):
+            blk = int(wl.block_tables[b, t // bs])
+            wl.k_cache[blk, :, t % bs] = NAN_CODE
+            wl.v_cache[blk, :, t % bs] = NAN_CODE
+        wl.block_tables[b, nb:] = 10 ** 6
+    used = set(wl.block_tables[wl.block_tables < wl.num_blocks].tolist())
+    for blk in range(wl.num_blocks):
+        if blk not in used:
+            wl.k_cache[blk] = NAN_CODE
+            wl.v_cache[blk] = NAN_CODE
+    d = dev(wl)
+    rc, info = pa.pa_plan(pa.params_for(d), block_size)
+    assert rc == pa.PA_OK and info.stages == 4
+    out = pa.decode(d)
+    assert_close(out.float().cpu().numpy(), ref, f"fp8 self-refill NaN codes BS={block_size}")
